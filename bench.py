@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Throughput of the jagged HSTU layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl ours|reference]
+
+A step is one forward of the whole workload: for the default workload the
+24-layer HSTU stack over 8 users x 8192 tokens (d 1024, 8 heads x 128, causal),
+i.e. every hot-path step (schedule, f1 GEMM, fused attention, LayerNorm-gate,
+f2 GEMM) for every layer.  The value is layer-tokens per second (tokens x
+layers / step time) over all ranks; each rank runs its own users (weak
+scaling, no collective on the data path).  Inputs are resident in HBM when
+the timed region starts; `e2e` repeats the measurement with the inputs copied
+from pinned host memory and the output copied back inside every step.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (one layer over one user's 4096-token causal
+prefix per step), in the same unit.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from jagged_pointwise_attention_hstu_b200 import workloads as wl  # noqa: E402
+
+METRIC = "HSTU layer fwd tokens/s (jagged) and attention TFLOP/s as % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def visible_pairs(lengths, ncand, mask):
+    total = 0
+    for n, c in zip(lengths, ncand):
+        n, c = int(n), int(c) if mask == "mfalcon" else 0
+        nh = n - c
+        total += nh * (nh + 1) // 2 + c * (nh + 1)
+    return total
+
+
+def workload_flops(w, batch):
+    T = batch.total_tokens
+    attn = 4 * w.head_dim * w.num_heads * visible_pairs(batch.lengths, batch.num_candidates, w.mask)
+    gemm = 10 * T * w.d_model * w.d_model
+    return attn, gemm
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(w, prefix, timed_layers=1):
+    """Times the fp64 oracle on one layer over user 0's causal prefix.
+
+    Returns (seconds, layer-tokens processed)."""
+    import oracle
+    batch = wl.make_batch(w, num_layers=1, num_users=1, max_len=prefix)
+    lp = batch.layers[0]
+    p = {k: np.asarray(getattr(lp, k), np.float32).astype(np.float64)
+         for k in ("b1", "b2", "rab_pos", "rab_time", "ln_gamma", "ln_beta")}
+    p["w1"] = wl.round_to_storage(lp.w1, w.compute).astype(np.float64)
+    p["w2"] = wl.round_to_storage(lp.w2, w.compute).astype(np.float64)
+    cfg = oracle.OracleConfig(d_model=w.d_model, num_heads=w.num_heads, head_dim=w.head_dim,
+                              pos_clamp=w.pos_clamp, time_buckets=w.time_buckets,
+                              time_log_div=w.time_log_div, n_norm=w.n_norm, ln_eps=w.ln_eps,
+                              mask=w.mask)
+    X = wl.round_to_storage(batch.x, w.storage).astype(np.float64)
+    t0 = time.perf_counter()
+    for _ in range(timed_layers):
+        oracle.hstu_layer(X, batch.seq_offsets, batch.timestamps, batch.num_candidates, p, cfg)
+    return time.perf_counter() - t0, batch.total_tokens * timed_layers
+
+
+def attention_traffic(kernel_src_hash, workload_index):
+    """dram bytes per attention launch from a committed ncu summary, if it was
+    taken on the current attention source; else None."""
+    path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        doc = json.load(f)
+    ent = doc.get(str(workload_index))
+    if not ent or ent.get("source_sha256") != kernel_src_hash:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for name in ("attn_tc.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "jagged_pointwise_attention_hstu_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = wl.WORKLOADS[args.workload]
+    prefix = 4096 if w.mask == "causal" else None
+    if prefix is None:
+        print(json.dumps({"impl": "reference", "unavailable": "reference sample defined for causal workloads"}))
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(w, prefix)
+    secs, units = 0.0, 0
+    for _ in range(args.steps):
+        s, u = oracle_sample(w, prefix)
+        secs += s
+        units += u
+    value = units / secs
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample": f"1 layer over user 0's first {prefix} tokens per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"1 layer x 1 user x {prefix}-token causal prefix per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from jagged_pointwise_attention_hstu_b200 import hstu, runtime
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    batch = wl.make_batch(w, seed_offset=rank)       # weak scaling: each rank its own users
+    L = len(batch.layers)
+    T = batch.total_tokens
+    cfg = runtime.config_for(w, T, batch.num_users)
+    handle = runtime.Handle(cfg, local)
+    db = runtime.to_device(batch, w.storage, w.compute, dev)
+    out = torch.empty_like(db.x)
+    mode = runtime.mask_mode_of(w)
+    stream = torch.cuda.current_stream(dev)
+    structs = [l.struct() for l in db.layers]
+
+    def step(x_in):
+        hstu.hstu_stack_forward(handle.h, x_in, T, db.seq_offsets, db.num_users, db.timestamps,
+                                structs, mode, db.num_candidates, out, stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step(db.x)
+    torch.cuda.synchronize(dev)
+    if handle.device_error():
+        raise RuntimeError("device error during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- device-resident timing
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    hstu.hstu_set_kernel_timing(handle.h, True)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            step(db.x)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = start.elapsed_time(end) / args.steps
+    ktimes = hstu.hstu_get_kernel_timing(handle.h)
+    hstu.hstu_set_kernel_timing(handle.h, False)
+    if handle.device_error():
+        raise RuntimeError("device error during the timed region")
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    units_per_rank = T * L
+    value = world * units_per_rank / (ms_max / 1e3)
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = db.x.cpu().pin_memory()
+        offs_host = db.seq_offsets.cpu().pin_memory()
+        ts_host = db.timestamps.cpu().pin_memory()
+        nc_host = db.num_candidates.cpu().pin_memory()
+        y_host = torch.empty_like(out, device="cpu").pin_memory()
+        x_dev = torch.empty_like(db.x)
+        h2d = x_host.numel() * x_host.element_size() + offs_host.numel() * 4 + ts_host.numel() * 8
+        if w.mask == "mfalcon":
+            h2d += nc_host.numel() * 4
+        d2h = y_host.numel() * y_host.element_size()
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            db.seq_offsets.copy_(offs_host, non_blocking=True)
+            db.timestamps.copy_(ts_host, non_blocking=True)
+            if w.mask == "mfalcon":
+                db.num_candidates.copy_(nc_host, non_blocking=True)
+            step(x_dev)
+            y_host.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = s2.elapsed_time(e2) / args.steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * units_per_rank / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": ms_e2e}
+
+    # ---------------- roofline of the dominant kernel (attention)
+    pk, pk_kind = peaks()
+    attn_flops, gemm_flops = workload_flops(w, batch)      # per layer
+    attn_ms, attn_n = ktimes["attention"]
+    f1_ms, f1_n = ktimes["f1"]
+    f2_ms, f2_n = ktimes["f2"]
+    ln_ms, ln_n = ktimes["ln_gate"]
+    attn_tflops = attn_flops / (attn_ms / attn_n / 1e3) / 1e12 if attn_n else None
+    peak_s = float(pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_b = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = attention_traffic(source_hash(), args.workload)
+    roofline = {"bound": "tensor", "kernel": "attention (fused jagged pointwise, tcgen05)",
+                "achieved": attn_tflops, "peak": peak_s, "unit": "TFLOP/s",
+                "frac": (attn_tflops / peak_s) if attn_tflops else None,
+                "peak_kind": f"{pk_kind} bf16_tflops_sustained (kernel timed inside a long step)",
+                "frac_of_burst_peak": (attn_tflops / peak_b) if attn_tflops else None,
+                "traffic": traffic,
+                "algorithmic_flops_per_launch": attn_flops,
+                "avg_launch_ms": attn_ms / attn_n if attn_n else None}
+    gemm_ms = (f1_ms + f2_ms) / max(f1_n, 1)
+    kernels = {k: {"total_ms": v[0], "launches": v[1]} for k, v in ktimes.items()}
+    launches = sum(v[1] for v in ktimes.values()) + ktimes["schedule"][1]   # rows + order kernels
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prefix = 8192 if w.mask == "causal" else None
+        if prefix is not None:
+            secs, units = oracle_sample(w, min(prefix, int(batch.lengths[0])))
+            cpu_baseline = {"value": units / secs, "unit": "tokens/s", "cores": blas_threads(),
+                            "kind": "oracle",
+                            "sample": f"1 layer x user 0 ({min(prefix, int(batch.lengths[0]))} "
+                                      f"tokens), fp64 numpy, {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "users_per_gpu": batch.num_users, "tokens_per_gpu": T,
+                   "layers": L, "d_model": w.d_model, "heads": w.num_heads,
+                   "head_dim": w.head_dim, "residual_stream": w.storage,
+                   "parallelism": f"dp{world} (users sharded, no collective)",
+                   "l2": "inputs larger than L2 (X fp32 256 MB, U|V|Q|K 512 MB per layer)",
+                   "unit_note": "tokens/s counts token-layers: tokens x layers / step time"},
+        "attention": {"tflops": attn_tflops, "pct_of_sustained_peak": 100 * attn_tflops / peak_s if attn_tflops else None,
+                      "pct_of_burst_peak": 100 * attn_tflops / peak_b if attn_tflops else None,
+                      "flops_per_layer": attn_flops},
+        "gemm": {"tflops": gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms else None,
+                 "flops_per_layer": gemm_flops},
+        "ln_gate": {"gbs": (T * w.d_model * (4 + 2 + 2)) / (ln_ms / ln_n / 1e3) / 1e9 if ln_n else None},
+        "kernels": kernels,
+        "roofline": roofline,
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    handle.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,218 @@
+/*
+ * hstu.h -- C ABI of the jagged HSTU layer forward for NVIDIA B200 (sm_100a).
+ *
+ * One HSTU layer (blog "Generative Recommendation 16: HSTU", section
+ * "HSTU Layer 到底改了什么", equations (1)-(3)):
+ *
+ *   (1)  U, V, Q, K = Split(SiLU(X W1^T + b1))            split order U, V, Q, K
+ *   (2)  O_i = sum_{j visible to i} SiLU(q_i . k_j + rab_pos[p(i,j)] + rab_time[t(i,j)]) v_j / n_norm
+ *   (3)  Y = (LayerNorm(O) (.) U) W2^T + b2 + X
+ *
+ * per head (heads are contiguous column blocks of width head_dim), with no
+ * softmax along the sequence (same blog, section "不对序列做 softmax").
+ * Batches are jagged: user b owns rows seq_offsets[b] .. seq_offsets[b+1]-1
+ * of every [T, *] tensor, with no padding ("Ragged/Jagged kernel" item of the
+ * same blog); no query ever sees another user's keys.
+ *
+ * Visibility (mask_mode):
+ *   HSTU_MASK_CAUSAL   key j visible to query i iff j <= i (same user).
+ *   HSTU_MASK_MFALCON  the last num_candidates[b] rows of user b are ranking
+ *                      candidates (ltzyclt blog on HSTU, section 5.2,
+ *                      "M-FALCON"): a candidate sees the user's whole history
+ *                      and itself, never another candidate; history rows are
+ *                      causal and never see candidates.  Every candidate sits
+ *                      at position n_h (the first position after the history),
+ *                      so results do not depend on how candidates are split
+ *                      into micro-batches.
+ * Bias buckets (the rab^{p,t} of equation (2); the rules are fixed by the
+ * layer configuration, not by the pages):
+ *   p(i,j) = clamp(pos(i) - j, 0, pos_clamp), pos(i) = i for history rows and
+ *            n_h for candidates (local indices inside the user);
+ *   t(i,j) = min(floor(ln(1 + max(ts_i - ts_j, 0)) / time_log_div), time_buckets - 1),
+ *            evaluated as that fp64 expression (the library turns it into an
+ *            exact integer threshold table once, at hstu_create).
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented "device" must be device memory of the handle's GPU
+ *     and 16-byte aligned; "host" pointers are ordinary host memory.
+ *   - The caller owns every input, output, weight and stream.  The handle owns
+ *     only its workspace (intermediates, scheduler tables, error word).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) except where stated.  A handle must not be used from two
+ *     streams at once: its workspace is shared by all of its calls.
+ *   - Host-detectable argument errors return a non-zero status before any
+ *     launch.  Problems that only the GPU can see (non-monotone seq_offsets,
+ *     seq_offsets[B] != T, num_candidates outside [0, length], timestamps that
+ *     decrease inside a user or lie outside [0, 2^62)) set the handle's device
+ *     error word and leave `out` undefined; hstu_get_device_error reads it.
+ *   - No call traps, aborts or exits the process.
+ */
+#ifndef HSTU_B200_H_
+#define HSTU_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,   /* a null pointer, bad size, bad enum, misaligned pointer */
+  HSTU_ERR_UNSUPPORTED = 2,   /* a shape the kernels do not implement (see hstu_create) */
+  HSTU_ERR_WORKSPACE = 3,     /* T or B above the max_tokens / max_users given at create */
+  HSTU_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  HSTU_ERR_DEVICE_CHECK = 5,  /* the GPU found invalid offsets / candidates / timestamps */
+  HSTU_ERR_TIMEOUT = 6        /* a kernel gave up a bounded wait (pipeline stall) */
+} hstu_status;
+
+typedef enum { HSTU_DTYPE_BF16 = 0, HSTU_DTYPE_FP32 = 1 } hstu_dtype;
+
+typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MFALCON = 1 } hstu_mask_mode;
+
+/* Device error bits reported through hstu_get_device_error. */
+#define HSTU_DEVERR_OFFSETS     0x1  /* seq_offsets not monotone, [0] != 0 or [B] != T */
+#define HSTU_DEVERR_CANDIDATES  0x2  /* num_candidates[b] < 0 or > length of user b */
+#define HSTU_DEVERR_TIMESTAMPS  0x4  /* decreasing inside a user, or outside [0, 2^62) */
+#define HSTU_DEVERR_TIMEOUT     0x8  /* a bounded pipeline wait expired */
+
+typedef struct {
+  int32_t d_model;          /* d = num_heads * head_dim; BF16 compute: 128, 256, 384, 512, 768
+                               or 1024; FP32 compute: also 64 */
+  int32_t num_heads;
+  int32_t head_dim;         /* BF16 compute: 64 or 128.  FP32 compute: 32, 64, 96 or 128 */
+  hstu_dtype io_dtype;      /* dtype of X (values) and Y (out) in HBM */
+  hstu_dtype compute_dtype; /* BF16: tcgen05 tensor-core path, bf16 operands, fp32 accumulate;
+                               FP32: fp32 SIMT path (every product and sum in fp32) */
+  int32_t n_norm;           /* > 0: fixed divisor; <= 0: the longest user of each call */
+  int32_t pos_buckets;      /* rows of rab_pos; pos_clamp < pos_buckets */
+  int32_t pos_clamp;        /* relative positions are clamped to [0, pos_clamp]; <= 4096 */
+  int32_t time_buckets;     /* rows of rab_time; 1..256 */
+  double time_log_div;      /* divisor of ln(1 + dt); > 0 */
+  float ln_eps;             /* LayerNorm epsilon (biased variance) */
+  int64_t max_tokens;       /* workspace sizing: largest T of any call; < 2^31 */
+  int32_t max_users;        /* workspace sizing: largest B of any call */
+} hstu_config;
+
+/* Parameters of one layer; all device pointers, caller-owned. */
+typedef struct {
+  const void* w1;        /* [4d, d] row-major (Linear layout), compute dtype */
+  const float* b1;       /* [4d] */
+  const void* w2;        /* [d, d] row-major, compute dtype */
+  const float* b2;       /* [d] */
+  const float* ln_gamma; /* [d] */
+  const float* ln_beta;  /* [d] */
+  const float* rab_pos;  /* [pos_buckets], shared by all heads */
+  const float* rab_time; /* [time_buckets], shared by all heads */
+} hstu_layer_weights;
+
+typedef struct hstu_handle_s hstu_handle;
+
+/* Validates `cfg` (host pointer), makes `device` current, allocates the
+ * workspace for max_tokens / max_users and uploads the time-bucket threshold
+ * table.  Synchronous.  *out receives the handle (NULL on error). */
+hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** out);
+
+/* Frees the workspace.  Synchronizes the device first.  NULL is a no-op. */
+hstu_status hstu_destroy(hstu_handle* h);
+
+/* One HSTU layer forward (equations (1)-(3) plus the residual).
+ *   values         device [T, d] io_dtype, the layer input X
+ *   total_tokens   T (0 <= T <= max_tokens)
+ *   seq_offsets    device int32 [num_users + 1], 0 = offsets[0] <= ... <= offsets[B] = T
+ *   num_users      B (0 <= B <= max_users); zero-length users are allowed
+ *   timestamps     device int64 [T] seconds, non-decreasing inside each user, in [0, 2^62)
+ *   weights        host pointer to device-pointer struct
+ *   mask_mode      HSTU_MASK_CAUSAL or HSTU_MASK_MFALCON
+ *   num_candidates device int32 [B]; required for MFALCON, ignored for CAUSAL
+ *   out            device [T, d] io_dtype; may alias `values` exactly
+ *   stream         cudaStream_t or NULL
+ * Returns HSTU_OK once every kernel is enqueued. */
+hstu_status hstu_layer_forward(hstu_handle* h, const void* values, int64_t total_tokens,
+                               const int32_t* seq_offsets, int32_t num_users,
+                               const int64_t* timestamps, const hstu_layer_weights* weights,
+                               hstu_mask_mode mask_mode, const int32_t* num_candidates,
+                               void* out, void* stream);
+
+/* A stack of num_layers layers (blog "Generative Recommendation 16: HSTU",
+ * section on the experiments: the largest configuration stacks 24 layers at
+ * length 8192 and embedding 1024).  layers: host array of num_layers structs.
+ * The residual stream stays in io_dtype between layers inside `out`; the
+ * jagged schedule is built once for all layers.  Same arguments otherwise. */
+hstu_status hstu_stack_forward(hstu_handle* h, const void* values, int64_t total_tokens,
+                               const int32_t* seq_offsets, int32_t num_users,
+                               const int64_t* timestamps, const hstu_layer_weights* layers,
+                               int32_t num_layers, hstu_mask_mode mask_mode,
+                               const int32_t* num_candidates, void* out, void* stream);
+
+/* Human-readable name of a status.  Never NULL. */
+const char* hstu_status_string(hstu_status s);
+
+/* Synchronizes the handle's device, then returns the device error word of the
+ * handle in *bits (HSTU_DEVERR_* flags; 0 = none) and clears it.  Returns
+ * HSTU_ERR_DEVICE_CHECK or HSTU_ERR_TIMEOUT when bits are set, else HSTU_OK. */
+hstu_status hstu_get_device_error(hstu_handle* h, int32_t* bits);
+
+/* Host only, no GPU needed: the exact integer threshold table of the time
+ * bucket rule.  out[k] (host int64 [num_buckets]) is the smallest gap dt >= 0
+ * whose bucket floor(ln(1 + dt) / div) (fp64) is >= k, capped at 2^62 when no
+ * gap below 2^62 reaches k; out[0] = 0.  bucket(dt) = #{k >= 1 : dt >= out[k]}. */
+hstu_status hstu_time_bucket_thresholds(double time_log_div, int32_t num_buckets, int64_t* out);
+
+/* ---- Kernel timing (CUDA events on the launching stream) ----
+ * When enabled, every kernel the handle launches is bracketed by a pair of
+ * CUDA events recorded on the call's stream; the pairs are read back by
+ * hstu_get_kernel_timing.  Kinds: 0 schedule (row facts + q-tile order),
+ * 1 fp32->bf16 cast of X, 2 f1 GEMM, 3 attention, 4 LayerNorm-gate, 5 f2 GEMM.
+ * At most 4096 launches are recorded between resets. */
+#define HSTU_KERNEL_KINDS 6
+
+/* Enables (1) or disables (0) the event pairs; enabling also resets them. */
+hstu_status hstu_set_kernel_timing(hstu_handle* h, int32_t enabled);
+
+/* Synchronizes on the recorded events and returns, per kind k < HSTU_KERNEL_KINDS,
+ * the summed duration in milliseconds (host double [HSTU_KERNEL_KINDS]) and the
+ * number of launches (host int64 [HSTU_KERNEL_KINDS]).  Either pointer may be NULL. */
+hstu_status hstu_get_kernel_timing(hstu_handle* h, double* total_ms, int64_t* launches);
+
+/* ---- Inspection entry points for tests (same library, same kernels) ---- */
+
+typedef enum {
+  HSTU_TENSOR_UVQK = 0,  /* [T, 4d] compute dtype: SiLU(f1(X)), columns U | V | Q | K */
+  HSTU_TENSOR_AV = 1,    /* [T, d] fp32: the attention output O of equation (2) */
+  HSTU_TENSOR_G = 2      /* [T, d] compute dtype: LayerNorm(O) (.) U */
+} hstu_tensor;
+
+/* Copies (device to device, async on `stream`) the first `bytes` of an
+ * intermediate of the handle's most recent forward into caller memory `dst`.
+ * For a stack, the intermediates are those of its last layer. */
+hstu_status hstu_copy_intermediate(hstu_handle* h, hstu_tensor which, void* dst, size_t bytes,
+                                   void* stream);
+
+/* Runs the attention kernel of the BF16 path in its recording variant on the
+ * handle's current Q/K/V workspace (zeroed first) and writes, for every
+ * (query i, key j) pair the kernel visits, its position bucket, time bucket
+ * and visibility into dense host-sized device arrays [T, T]: pidx_out and
+ * tidx_out int32, vis_out uint8.  Pairs the kernel never visits (tiles it
+ * skips) keep the caller's contents.  Only for small batches: T <= 4096.
+ * Synchronous. */
+hstu_status hstu_debug_attention_buckets(hstu_handle* h, int64_t total_tokens,
+                                         const int32_t* seq_offsets, int32_t num_users,
+                                         const int64_t* timestamps, hstu_mask_mode mask_mode,
+                                         const int32_t* num_candidates, int32_t* pidx_out,
+                                         int32_t* tidx_out, uint8_t* vis_out);
+
+/* One 128 x n x k tile product on the tensor cores, to check the operand
+ * layouts the kernels use: mode 0 = A[128,k] K-major (smem) x B[n,k] K-major
+ * (smem); mode 1 = B given as [k, n] (N-major, smem); mode 2 = A staged in
+ * tensor memory, B [k, n] N-major.  a, b bf16 device, c fp32 device [128, n].
+ * n in {64, 128, 256} (mode >= 1: 64 or 128), k in {64, 128}.  Synchronous. */
+hstu_status hstu_debug_umma_tile(int32_t mode, const void* a, const void* b, float* c, int32_t n,
+                                 int32_t k);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_B200_H_ */

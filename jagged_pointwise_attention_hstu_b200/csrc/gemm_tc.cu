@@ -1,0 +1,286 @@
+// f1 and f2 of the HSTU layer as tcgen05 GEMMs over the jagged token axis.
+//
+//   f1:  UVQK = SiLU(X W1^T + b1)      (blog "Generative Recommendation 16:
+//        HSTU", section "HSTU Layer 到底改了什么", equation (1); the split into
+//        U, V, Q, K is the column order of the output, so it costs nothing)
+//   f2:  Y = G W2^T + b2 + X           (equation (3) plus the residual)
+//
+// The token axis is never padded: M = T rows ("fully ragged GEMM", item 1 of
+// the same blog's list of extra pieces); TMA zero-fills rows past T and the
+// epilogue masks them.
+//
+// Persistent, warp-specialised: warp 0 streams A/B k-blocks with TMA into a
+// 4-stage ring, warp 1 issues 128 x BN x 16 MMAs into one of two tensor-memory
+// accumulators, warps 2-5 drain the other accumulator through the fused
+// epilogue, so the epilogue of tile t overlaps the MMAs of tile t+1.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace hstu {
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 4;
+constexpr int kBK = 64;   // one 128-byte swizzle row of bf16
+
+struct GemmParams {
+  int64_t M;
+  int N, K;
+  int epi;              // Epi
+  const float* bias;
+  void* out;
+  const void* residual;
+  int io_fp32;
+  int32_t* error;
+};
+
+template <int BN>
+struct GemmLayout {
+  static constexpr uint32_t kABytes = 128 * kBK * 2;
+  static constexpr uint32_t kBBytes = BN * kBK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kBarOffset = kStages * kStageBytes;
+  static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
+};
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
+                   const __grid_constant__ CUtensorMap tma_b, const GemmParams p) {
+  using L = GemmLayout<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tma_a);
+    prefetch_tmap(&tma_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t m_tiles = (p.M + 127) / 128;
+  const int n_tiles = p.N / BN;
+  const int64_t total = m_tiles * n_tiles;
+  const int kblocks = p.K / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued_phase[kStages];
+      bool issued[kStages];
+      for (int s = 0; s < kStages; ++s) issued[s] = false, issued_phase[s] = 0;
+      for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const int64_t mt = t / n_tiles;
+        const int nt = int(t % n_tiles);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          tma_load_2d(sa, &tma_a, &full[stage], kb * kBK, int32_t(mt * 128));
+          tma_load_2d(sa + L::kABytes, &tma_b, &full[stage], kb * kBK, nt * BN);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      // every load this thread issued has landed before the CTA may exit
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s]) mbar_wait(&full[s], issued_phase[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool any = false;
+      for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
+          const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            umma_ss(d_tmem, desc_sw128(a_addr + k * 32, 16, 1024),
+                    desc_sw128(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[stage]);
+          any = true;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        umma_commit(&acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      if (any) {
+        umma_commit(drain);
+        mbar_wait(drain, 0);
+      }
+    }
+  } else {
+    // epilogue: warps 2..5, each owns the 32 tensor-memory lanes of its quarter
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint32_t acc = 0, acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+      if (*abort_flag) break;
+      if (!mbar_wait(&acc_full[acc], acc_phase)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int64_t mt = t / n_tiles;
+      const int nt = int(t % n_tiles);
+      const int64_t grow = mt * 128 + row;
+      const bool valid = grow < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + acc * BN + c + (uint32_t(q * 32) << 16), r);
+        tmem_ld_wait();
+        if (!valid) continue;
+        const int col0 = nt * BN + c;
+        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 bb = __ldg(b4 + e);
+          v[4 * e + 0] = __uint_as_float(r[4 * e + 0]) + bb.x;
+          v[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y;
+          v[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z;
+          v[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w;
+        }
+        if (p.epi == int(Epi::kSiluSplit)) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                                                grow * int64_t(p.N) + col0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 o;
+            o.x = pack_bf16x2(silu_f(v[8 * e + 0]), silu_f(v[8 * e + 1]));
+            o.y = pack_bf16x2(silu_f(v[8 * e + 2]), silu_f(v[8 * e + 3]));
+            o.z = pack_bf16x2(silu_f(v[8 * e + 4]), silu_f(v[8 * e + 5]));
+            o.w = pack_bf16x2(silu_f(v[8 * e + 6]), silu_f(v[8 * e + 7]));
+            dst[e] = o;
+          }
+        } else if (p.io_fp32) {
+          const float4* res = reinterpret_cast<const float4*>(
+              static_cast<const float*>(p.residual) + grow * int64_t(p.N) + col0);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) +
+                                                  grow * int64_t(p.N) + col0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 x = res[e];
+            dst[e] = make_float4(v[4 * e + 0] + x.x, v[4 * e + 1] + x.y, v[4 * e + 2] + x.z,
+                                 v[4 * e + 3] + x.w);
+          }
+        } else {
+          const uint4* res = reinterpret_cast<const uint4*>(
+              static_cast<const uint16_t*>(p.residual) + grow * int64_t(p.N) + col0);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                                                grow * int64_t(p.N) + col0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint4 x = res[e];
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+            uint32_t os[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float lo = __uint_as_float(xs[w] << 16);
+              const float hi = __uint_as_float(xs[w] & 0xFFFF0000u);
+              os[w] = pack_bf16x2(v[8 * e + 2 * w] + lo, v[8 * e + 2 * w + 1] + hi);
+            }
+            dst[e] = make_uint4(os[0], os[1], os[2], os[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.error, HSTU_DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
+  using L = GemmLayout<BN>;
+  CUtensorMap ta, tb;
+  if (!make_tmap_2d_bf16(&ta, a.a, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K) * 2, kBK, 128))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK, BN))
+    return cudaErrorInvalidValue;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(L::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  GemmParams p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.epi = int(a.epi);
+  p.bias = a.bias;
+  p.out = a.out;
+  p.residual = a.residual;
+  p.io_fp32 = a.io_fp32;
+  p.error = error;
+  const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
+  const int grid = int(tiles < num_sms ? tiles : num_sms);
+  gemm_tc_kernel<BN><<<grid, 192, L::kSmemBytes, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
+  if (a.M <= 0) return cudaSuccess;
+  if (a.K % kBK != 0 || a.N % 128 != 0) return cudaErrorInvalidValue;
+  if (a.N % 256 == 0) return launch_bn<256>(a, num_sms, st, error);
+  return launch_bn<128>(a, num_sms, st, error);
+}
+
+}  // namespace hstu

@@ -1,0 +1,499 @@
+// C ABI of the jagged HSTU layer forward: argument checks, workspace, tensor
+// maps and the launch sequence of one layer / one stack.  Every step of the
+// forward runs in this library's kernels; nothing here computes layer math on
+// the host except the integer threshold table of the time-bucket rule.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "internal.h"
+
+using hstu::Workspace;
+
+namespace hstu {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bucket index of gap dt under the fp64 rule floor(ln(1 + dt) / div)
+int64_t fp64_bucket(int64_t dt, double div) {
+  if (dt <= 0) return 0;
+  return static_cast<int64_t>(floor(log(1.0 + static_cast<double>(dt)) / div));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename T>
+cudaError_t alloc(T** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  return cudaMalloc(reinterpret_cast<void**>(p), bytes);
+}
+
+size_t elem_size(hstu_dtype t) { return t == HSTU_DTYPE_BF16 ? 2 : 4; }
+
+}  // namespace
+
+bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr || outer == 0 || inner == 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace hstu
+
+extern "C" {
+
+const char* hstu_status_string(hstu_status s) {
+  switch (s) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED";
+    case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA";
+    case HSTU_ERR_DEVICE_CHECK: return "HSTU_ERR_DEVICE_CHECK";
+    case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT";
+  }
+  return "HSTU_ERR_UNKNOWN";
+}
+
+hstu_status hstu_time_bucket_thresholds(double div, int32_t nb, int64_t* out) {
+  if (out == nullptr || !(div > 0.0) || nb < 1 || nb > 256) return HSTU_ERR_INVALID_ARG;
+  out[0] = 0;
+  for (int32_t k = 1; k < nb; ++k) {
+    // smallest dt in [0, 2^62] with bucket(dt) >= k; the rule is monotone in dt
+    int64_t lo = 0, hi = hstu::kMaxTimestamp;
+    if (hstu::fp64_bucket(hi, div) < k) {
+      out[k] = hstu::kMaxTimestamp;
+      continue;
+    }
+    while (lo < hi) {
+      const int64_t mid = lo + (hi - lo) / 2;
+      if (hstu::fp64_bucket(mid, div) >= k) hi = mid; else lo = mid + 1;
+    }
+    out[k] = lo;
+  }
+  return HSTU_OK;
+}
+
+hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** out) {
+  if (out == nullptr || cfg == nullptr) return HSTU_ERR_INVALID_ARG;
+  *out = nullptr;
+  const hstu_config& c = *cfg;
+  if (c.d_model <= 0 || c.num_heads <= 0 || c.head_dim <= 0 ||
+      c.d_model != c.num_heads * c.head_dim)
+    return HSTU_ERR_INVALID_ARG;
+  if ((c.io_dtype != HSTU_DTYPE_BF16 && c.io_dtype != HSTU_DTYPE_FP32) ||
+      (c.compute_dtype != HSTU_DTYPE_BF16 && c.compute_dtype != HSTU_DTYPE_FP32))
+    return HSTU_ERR_INVALID_ARG;
+  if (c.pos_buckets < 1 || c.pos_clamp < 0 || c.pos_clamp >= c.pos_buckets) return HSTU_ERR_INVALID_ARG;
+  if (c.time_buckets < 1 || c.time_buckets > 256 || !(c.time_log_div > 0.0)) return HSTU_ERR_INVALID_ARG;
+  if (!(c.ln_eps >= 0.0f) || c.max_tokens < 0 || c.max_tokens >= (int64_t(1) << 31) ||
+      c.max_users < 0)
+    return HSTU_ERR_INVALID_ARG;
+  if (c.pos_clamp > 4096) return HSTU_ERR_UNSUPPORTED;
+  const int d = c.d_model;
+  const bool d_ok = d == 64 || (d % 128 == 0 && d <= 1024 && d != 896 && d != 640);
+  if (!d_ok) return HSTU_ERR_UNSUPPORTED;
+  if (c.compute_dtype == HSTU_DTYPE_BF16) {
+    if (c.head_dim != 64 && c.head_dim != 128) return HSTU_ERR_UNSUPPORTED;
+    if (d % 128 != 0) return HSTU_ERR_UNSUPPORTED;
+  } else {
+    if (c.io_dtype != HSTU_DTYPE_FP32) return HSTU_ERR_UNSUPPORTED;
+    if (c.head_dim % 32 != 0 || c.head_dim > 128) return HSTU_ERR_UNSUPPORTED;
+  }
+  if (cudaSetDevice(device) != cudaSuccess) return HSTU_ERR_CUDA;
+  hstu_handle* h = new (std::nothrow) hstu_handle_s();
+  if (h == nullptr) return HSTU_ERR_CUDA;
+  h->cfg = c;
+  h->device = device;
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, device);
+  if (hstu_time_bucket_thresholds(c.time_log_div, c.time_buckets, h->thresholds_host) != HSTU_OK) {
+    delete h;
+    return HSTU_ERR_INVALID_ARG;
+  }
+  const size_t T = size_t(c.max_tokens);
+  const size_t cs = hstu::elem_size(c.compute_dtype);
+  const size_t nqt = (T + hstu::kTile - 1) / hstu::kTile + 1;
+  Workspace& ws = h->ws;
+  cudaError_t e = cudaSuccess;
+  if (c.compute_dtype == HSTU_DTYPE_BF16 && c.io_dtype == HSTU_DTYPE_FP32)
+    e = hstu::alloc(&ws.xb, T * d * 2);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.uvqk, T * 4 * d * cs);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.av, T * d * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.g, T * d * cs);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.rows, T * sizeof(hstu::RowInfo));
+  if (e == cudaSuccess) e = hstu::alloc(&ws.qtile_order, nqt * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.qtile_cost, nqt * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.counters, 16);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.error, 16);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.thresholds, 256 * 8);
+  if (e == cudaSuccess) e = cudaMemset(ws.error, 0, 16);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(ws.thresholds, h->thresholds_host, size_t(c.time_buckets) * 8,
+                   cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    hstu_destroy(h);
+    return HSTU_ERR_CUDA;
+  }
+  *out = h;
+  return HSTU_OK;
+}
+
+hstu_status hstu_destroy(hstu_handle* h) {
+  if (h == nullptr) return HSTU_OK;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  Workspace& ws = h->ws;
+  void* ptrs[] = {ws.xb, ws.uvqk, ws.av, ws.g, ws.rows, ws.qtile_order, ws.qtile_cost,
+                  ws.counters, ws.error, ws.thresholds};
+  for (void* p : ptrs)
+    if (p != nullptr) cudaFree(p);
+  if (h->timer.created)
+    for (int i = 0; i < 2 * hstu::KernelTimer::kMax; ++i) cudaEventDestroy(h->timer.ev[i]);
+  delete h;
+  return HSTU_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+enum Kind { kSchedule = 0, kCast = 1, kF1 = 2, kAttention = 3, kLnGate = 4, kF2 = 5 };
+
+// Brackets one launch with a pair of events when the handle's timer is on.
+struct Timed {
+  hstu::KernelTimer* t;
+  cudaStream_t st;
+  int idx = -1;
+  Timed(hstu_handle* h, int kind, cudaStream_t s) : t(&h->timer), st(s) {
+    if (t->enabled && t->count < hstu::KernelTimer::kMax) {
+      idx = t->count++;
+      t->kind[idx] = kind;
+      cudaEventRecord(t->ev[2 * idx], st);
+    }
+  }
+  ~Timed() {
+    if (idx >= 0) cudaEventRecord(t->ev[2 * idx + 1], st);
+  }
+};
+
+hstu_status check_common(hstu_handle* h, const void* values, int64_t T, const int32_t* offsets,
+                         int32_t B, const int64_t* ts, hstu_mask_mode mode,
+                         const int32_t* ncand, const void* out) {
+  if (h == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (T < 0 || B < 0) return HSTU_ERR_INVALID_ARG;
+  if (T > h->cfg.max_tokens || B > h->cfg.max_users) return HSTU_ERR_WORKSPACE;
+  if (mode != HSTU_MASK_CAUSAL && mode != HSTU_MASK_MFALCON) return HSTU_ERR_INVALID_ARG;
+  if (B == 0 && T != 0) return HSTU_ERR_INVALID_ARG;
+  if (offsets == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (values == nullptr || out == nullptr || ts == nullptr) return HSTU_ERR_INVALID_ARG;
+    if (!hstu::aligned16(values) || !hstu::aligned16(out) || !hstu::aligned16(ts))
+      return HSTU_ERR_INVALID_ARG;
+  }
+  if (mode == HSTU_MASK_MFALCON && B > 0 && ncand == nullptr) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+hstu_status check_weights(const hstu_layer_weights* w) {
+  if (w == nullptr) return HSTU_ERR_INVALID_ARG;
+  const void* ps[] = {w->w1, w->b1, w->w2, w->b2, w->ln_gamma, w->ln_beta, w->rab_pos, w->rab_time};
+  for (const void* p : ps)
+    if (p == nullptr || !hstu::aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+// One layer after the schedule is built: f1 -> attention -> LN (.) U -> f2.
+hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* ts,
+                      const hstu_layer_weights* w, void* out, cudaStream_t st) {
+  const hstu_config& c = h->cfg;
+  Workspace& ws = h->ws;
+  const int d = c.d_model;
+  const bool f32 = c.compute_dtype == HSTU_DTYPE_FP32;
+  const bool io32 = c.io_dtype == HSTU_DTYPE_FP32;
+  cudaError_t e = cudaSuccess;
+  hstu::AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.uvqk = ws.uvqk;
+  a.av = ws.av;
+  a.rows = ws.rows;
+  a.order = ws.qtile_order;
+  a.ts = ts;
+  a.thresholds = ws.thresholds;
+  a.rab_pos = w->rab_pos;
+  a.rab_time = w->rab_time;
+  a.counters = ws.counters;
+  a.error = ws.error;
+  a.T = T;
+  a.d = d;
+  a.H = c.num_heads;
+  a.hd = c.head_dim;
+  a.pos_clamp = c.pos_clamp;
+  a.time_buckets = c.time_buckets;
+  a.n_norm_fixed = c.n_norm;
+  a.num_qtiles = int((T + hstu::kTile - 1) / hstu::kTile);
+  if (f32) {
+    {
+      Timed tm(h, kF1, st);
+      e = hstu::launch_gemm_f32(static_cast<const float*>(x), static_cast<const float*>(w->w1), T,
+                                4 * d, d, hstu::Epi::kSiluSplit, w->b1,
+                                static_cast<float*>(ws.uvqk), nullptr, st);
+    }
+    if (e == cudaSuccess) {
+      Timed tm(h, kAttention, st);
+      e = hstu::launch_attention_f32(a, st);
+    }
+    if (e == cudaSuccess) {
+      Timed tm(h, kLnGate, st);
+      e = hstu::launch_ln_gate(ws.av, ws.uvqk, ws.g, w->ln_gamma, w->ln_beta, T, d, c.ln_eps, 1, st);
+    }
+    if (e == cudaSuccess) {
+      Timed tm(h, kF2, st);
+      e = hstu::launch_gemm_f32(static_cast<const float*>(ws.g), static_cast<const float*>(w->w2),
+                                T, d, d, hstu::Epi::kBiasResidual, w->b2, static_cast<float*>(out),
+                                static_cast<const float*>(x), st);
+    }
+    return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  }
+  const void* xa = x;
+  if (io32) {
+    Timed tm(h, kCast, st);
+    e = hstu::launch_cast_bf16(static_cast<const float*>(x), ws.xb, T * d, st);
+    xa = ws.xb;
+  }
+  hstu::GemmArgs g1;
+  g1.a = xa;
+  g1.b = w->w1;
+  g1.M = T;
+  g1.N = 4 * d;
+  g1.K = d;
+  g1.epi = hstu::Epi::kSiluSplit;
+  g1.bias = w->b1;
+  g1.out = ws.uvqk;
+  g1.residual = nullptr;
+  g1.io_fp32 = 0;
+  if (e == cudaSuccess) {
+    Timed tm(h, kF1, st);
+    e = hstu::launch_gemm_tc(g1, h->num_sms, st, ws.error);
+  }
+  if (e == cudaSuccess) {
+    Timed tm(h, kAttention, st);
+    e = hstu::launch_attention_tc(a, st, false);
+  }
+  if (e == cudaSuccess) {
+    Timed tm(h, kLnGate, st);
+    e = hstu::launch_ln_gate(ws.av, ws.uvqk, ws.g, w->ln_gamma, w->ln_beta, T, d, c.ln_eps, 0, st);
+  }
+  hstu::GemmArgs g2;
+  g2.a = ws.g;
+  g2.b = w->w2;
+  g2.M = T;
+  g2.N = d;
+  g2.K = d;
+  g2.epi = hstu::Epi::kBiasResidual;
+  g2.bias = w->b2;
+  g2.out = out;
+  g2.residual = x;
+  g2.io_fp32 = io32 ? 1 : 0;
+  if (e == cudaSuccess) {
+    Timed tm(h, kF2, st);
+    e = hstu::launch_gemm_tc(g2, h->num_sms, st, ws.error);
+  }
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+hstu_status hstu_layer_forward(hstu_handle* h, const void* values, int64_t T,
+                               const int32_t* offsets, int32_t B, const int64_t* ts,
+                               const hstu_layer_weights* w, hstu_mask_mode mode,
+                               const int32_t* ncand, void* out, void* stream) {
+  return hstu_stack_forward(h, values, T, offsets, B, ts, w, 1, mode, ncand, out, stream);
+}
+
+hstu_status hstu_stack_forward(hstu_handle* h, const void* values, int64_t T,
+                               const int32_t* offsets, int32_t B, const int64_t* ts,
+                               const hstu_layer_weights* layers, int32_t num_layers,
+                               hstu_mask_mode mode, const int32_t* ncand, void* out,
+                               void* stream) {
+  hstu_status s = check_common(h, values, T, offsets, B, ts, mode, ncand, out);
+  if (s != HSTU_OK) return s;
+  if (layers == nullptr || num_layers < 1) return HSTU_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    s = check_weights(&layers[l]);
+    if (s != HSTU_OK) return s;
+  }
+  if (T == 0) return HSTU_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    Timed tm(h, kSchedule, st);
+    if (hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+  }
+  h->last_T = T;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    const void* x = (l == 0) ? values : out;
+    s = run_layer(h, x, T, ts, &layers[l], out, st);
+    if (s != HSTU_OK) return s;
+  }
+  return HSTU_OK;
+}
+
+hstu_status hstu_get_device_error(hstu_handle* h, int32_t* bits) {
+  if (h == nullptr || bits == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return HSTU_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, h->ws.error, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaMemset(h->ws.error, 0, 4) != cudaSuccess) return HSTU_ERR_CUDA;
+  *bits = v;
+  if (v & HSTU_DEVERR_TIMEOUT) return HSTU_ERR_TIMEOUT;
+  return v ? HSTU_ERR_DEVICE_CHECK : HSTU_OK;
+}
+
+hstu_status hstu_copy_intermediate(hstu_handle* h, hstu_tensor which, void* dst, size_t bytes,
+                                   void* stream) {
+  if (h == nullptr || dst == nullptr) return HSTU_ERR_INVALID_ARG;
+  const size_t T = size_t(h->cfg.max_tokens), d = size_t(h->cfg.d_model);
+  const size_t cs = hstu::elem_size(h->cfg.compute_dtype);
+  const void* src = nullptr;
+  size_t cap = 0;
+  switch (which) {
+    case HSTU_TENSOR_UVQK: src = h->ws.uvqk; cap = T * 4 * d * cs; break;
+    case HSTU_TENSOR_AV: src = h->ws.av; cap = T * d * 4; break;
+    case HSTU_TENSOR_G: src = h->ws.g; cap = T * d * cs; break;
+    default: return HSTU_ERR_INVALID_ARG;
+  }
+  if (bytes > cap) return HSTU_ERR_INVALID_ARG;
+  if (bytes == 0) return HSTU_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice,
+                         static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? HSTU_OK
+             : HSTU_ERR_CUDA;
+}
+
+hstu_status hstu_debug_attention_buckets(hstu_handle* h, int64_t T, const int32_t* offsets,
+                                         int32_t B, const int64_t* ts, hstu_mask_mode mode,
+                                         const int32_t* ncand, int32_t* pidx_out,
+                                         int32_t* tidx_out, uint8_t* vis_out) {
+  hstu_status s = check_common(h, reinterpret_cast<const void*>(16), T, offsets, B, ts, mode, ncand,
+                               reinterpret_cast<const void*>(16));
+  if (s != HSTU_OK) return s;
+  if (h->cfg.compute_dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (T > 4096 || pidx_out == nullptr || tidx_out == nullptr || vis_out == nullptr)
+    return HSTU_ERR_INVALID_ARG;
+  if (T == 0) return HSTU_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu_config& c = h->cfg;
+  const int d = c.d_model;
+  // zero Q/K/V so that the kernel reads defined values; biases from zero tables
+  float* zeros = nullptr;
+  if (cudaMalloc(&zeros, size_t(c.pos_buckets + c.time_buckets) * 4) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  cudaMemset(zeros, 0, size_t(c.pos_buckets + c.time_buckets) * 4);
+  cudaMemset(h->ws.uvqk, 0, size_t(T) * 4 * d * 2);
+  cudaError_t e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, 0);
+  hstu::AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.uvqk = h->ws.uvqk;
+  a.av = h->ws.av;
+  a.rows = h->ws.rows;
+  a.order = h->ws.qtile_order;
+  a.ts = ts;
+  a.thresholds = h->ws.thresholds;
+  a.rab_pos = zeros;
+  a.rab_time = zeros + c.pos_buckets;
+  a.counters = h->ws.counters;
+  a.error = h->ws.error;
+  a.T = T;
+  a.d = d;
+  a.H = c.num_heads;
+  a.hd = c.head_dim;
+  a.pos_clamp = c.pos_clamp;
+  a.time_buckets = c.time_buckets;
+  a.n_norm_fixed = c.n_norm;
+  a.num_qtiles = int((T + hstu::kTile - 1) / hstu::kTile);
+  a.dump_pidx = pidx_out;
+  a.dump_tidx = tidx_out;
+  a.dump_vis = vis_out;
+  if (e == cudaSuccess) e = hstu::launch_attention_tc(a, 0, true);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(zeros);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status hstu_set_kernel_timing(hstu_handle* h, int32_t enabled) {
+  if (h == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  hstu::KernelTimer& t = h->timer;
+  if (enabled && !t.created) {
+    for (int i = 0; i < 2 * hstu::KernelTimer::kMax; ++i)
+      if (cudaEventCreate(&t.ev[i]) != cudaSuccess) return HSTU_ERR_CUDA;
+    t.created = true;
+  }
+  t.enabled = enabled != 0;
+  if (t.enabled) t.count = 0;
+  return HSTU_OK;
+}
+
+hstu_status hstu_get_kernel_timing(hstu_handle* h, double* total_ms, int64_t* launches) {
+  if (h == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  double ms[HSTU_KERNEL_KINDS] = {0};
+  int64_t n[HSTU_KERNEL_KINDS] = {0};
+  const hstu::KernelTimer& t = h->timer;
+  for (int i = 0; i < t.count; ++i) {
+    if (cudaEventSynchronize(t.ev[2 * i + 1]) != cudaSuccess) return HSTU_ERR_CUDA;
+    float e = 0.f;
+    if (cudaEventElapsedTime(&e, t.ev[2 * i], t.ev[2 * i + 1]) != cudaSuccess) return HSTU_ERR_CUDA;
+    ms[t.kind[i]] += e;
+    n[t.kind[i]] += 1;
+  }
+  for (int k = 0; k < HSTU_KERNEL_KINDS; ++k) {
+    if (total_ms != nullptr) total_ms[k] = ms[k];
+    if (launches != nullptr) launches[k] = n[k];
+  }
+  return HSTU_OK;
+}
+
+hstu_status hstu_debug_umma_tile(int32_t mode, const void* a, const void* b, float* c, int32_t n,
+                                 int32_t k) {
+  if (a == nullptr || b == nullptr || c == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 2 || (k != 64 && k != 128)) return HSTU_ERR_INVALID_ARG;
+  if (mode == 0 && n != 64 && n != 128 && n != 256) return HSTU_ERR_INVALID_ARG;
+  if (mode != 0 && n != 64 && n != 128) return HSTU_ERR_INVALID_ARG;
+  const cudaError_t e = hstu::run_umma_tile(mode, a, b, c, n, k);
+  if (e == cudaErrorLaunchTimeout) return HSTU_ERR_TIMEOUT;
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+}  // extern "C"

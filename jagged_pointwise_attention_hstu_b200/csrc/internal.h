@@ -1,0 +1,128 @@
+// Internal declarations shared by the C-ABI implementation and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hstu.h"
+
+namespace hstu {
+
+constexpr int kTile = 128;            // query / key rows per attention tile, GEMM BM
+constexpr int64_t kMaxTimestamp = int64_t(1) << 62;
+
+// Per-token facts the attention kernels need, built by the scheduler.
+//   lo: first row of the token's user; hi: one past the last key the token may
+//   aggregate besides itself (i + 1 for history rows, n_h start for candidates);
+//   pos: the position anchor (i for history rows, the user's history end for
+//   candidates), so the position bucket of key j is clamp(pos - j, 0, clamp).
+struct RowInfo {
+  int32_t lo, hi, pos, user;
+};
+
+struct Workspace {
+  void* xb = nullptr;          // [T, d] bf16: X cast for the GEMM when io is fp32
+  void* uvqk = nullptr;        // [T, 4d] compute dtype
+  float* av = nullptr;         // [T, d] fp32
+  void* g = nullptr;           // [T, d] compute dtype
+  RowInfo* rows = nullptr;     // [T]
+  int32_t* qtile_order = nullptr;  // [ceil(T / 128)] q-tiles by descending cost
+  int32_t* qtile_cost = nullptr;   // [ceil(T / 128)]
+  int32_t* counters = nullptr;     // [4]: n_norm, max cost, scratch
+  int32_t* error = nullptr;        // device error word
+  int64_t* thresholds = nullptr;   // [time_buckets] time-bucket thresholds
+};
+
+}  // namespace hstu
+
+namespace hstu {
+// CUDA-event pairs around every kernel launch of a handle (off by default).
+struct KernelTimer {
+  static constexpr int kMax = 4096;
+  bool enabled = false;
+  int count = 0;
+  int kind[kMax];
+  cudaEvent_t ev[2 * kMax];
+  bool created = false;
+};
+}  // namespace hstu
+
+struct hstu_handle_s {
+  hstu_config cfg;
+  hstu::KernelTimer timer;
+  int device = 0;
+  int num_sms = 148;
+  hstu::Workspace ws;
+  int64_t last_T = 0;
+  int64_t thresholds_host[256];
+};
+
+namespace hstu {
+
+// sched.cu
+cudaError_t launch_schedule(const hstu_handle_s* h, int64_t T, const int32_t* offsets, int32_t B,
+                            const int64_t* ts, int mask_mode, const int32_t* ncand,
+                            cudaStream_t st);
+cudaError_t launch_cast_bf16(const float* x, void* xb, int64_t n, cudaStream_t st);
+
+// gemm_tc.cu
+enum class Epi { kSiluSplit = 0, kBiasResidual = 1 };
+struct GemmArgs {
+  const void* a;        // [M, K] bf16
+  const void* b;        // [N, K] bf16
+  int64_t M;
+  int N, K;
+  Epi epi;
+  const float* bias;    // [N]
+  // kSiluSplit: out bf16 [M, N]
+  // kBiasResidual: out = acc + bias + residual (io dtype), residual may alias out
+  void* out;
+  const void* residual;
+  int io_fp32;
+};
+cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error);
+
+// attn_tc.cu
+struct AttnArgs {
+  const void* uvqk;          // [T, 4d] bf16
+  float* av;                 // [T, d] fp32
+  const RowInfo* rows;
+  const int32_t* order;      // q-tile order
+  const int64_t* ts;
+  const int64_t* thresholds; // [time_buckets]
+  const float* rab_pos;
+  const float* rab_time;
+  const int32_t* counters;   // [0] = n_norm
+  int32_t* error;
+  int64_t T;
+  int d, H, hd;
+  int pos_clamp, time_buckets;
+  int n_norm_fixed;          // > 0: use it; else counters[0]
+  int num_qtiles;
+  // recording variant
+  int32_t* dump_pidx;
+  int32_t* dump_tidx;
+  uint8_t* dump_vis;
+};
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t st, bool record);
+
+// ln_gate.cu
+cudaError_t launch_ln_gate(const float* av, const void* uvqk, void* g, const float* gamma,
+                           const float* beta, int64_t T, int d, float eps, int compute_fp32,
+                           cudaStream_t st);
+
+// simt_fp32.cu
+cudaError_t launch_gemm_f32(const float* a, const float* b, int64_t M, int N, int K, Epi epi,
+                            const float* bias, float* out, const float* residual,
+                            cudaStream_t st);
+cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st);
+
+// umma_check.cu
+cudaError_t run_umma_tile(int mode, const void* a, const void* b, float* c, int n, int k);
+
+// tensor maps (hstu_api.cu)
+bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace hstu

@@ -1,0 +1,86 @@
+"""The C-ABI library loads and exports every declared entry point; host-side
+logic (argument checks, the time-bucket threshold table) runs without a GPU."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from jagged_pointwise_attention_hstu_b200 import build, hstu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return hstu.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = hstu.declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert hstu.status_string(s).startswith("HSTU_")
+    assert hstu.status_string(99) == "HSTU_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("div,nb", [(0.301, 128), (0.5, 64), (0.1, 256)])
+def test_time_thresholds_reproduce_the_bucket_rule(lib, div, nb):
+    """The library's integer thresholds give exactly the oracle's fp64 buckets."""
+    thr = np.array(hstu.hstu_time_bucket_thresholds(div, nb), dtype=np.int64)
+    assert thr[0] == 0 and np.all(np.diff(thr) >= 0)
+    reach = thr < 2 ** 62
+    k = np.nonzero(reach)[0][1:]
+    # at each threshold the bucket reaches k; one second earlier it is below k
+    assert np.all(oracle.time_bucket(thr[k], div, nb) >= k)
+    assert np.all(oracle.time_bucket(thr[k] - 1, div, nb) < k)
+    # bucket(dt) = #{k >= 1 : dt >= thr[k]} on a dense and a wide sample of gaps
+    rng = np.random.default_rng(0)
+    dts = np.concatenate([np.arange(0, 5000), rng.integers(0, 2 ** 40, 20000),
+                          np.unique(thr[reach]) + 1, np.unique(thr[reach]) - 1])
+    dts = dts[dts >= 0]
+    mine = (dts[:, None] >= thr[None, 1:]).sum(axis=1)
+    assert np.array_equal(mine, oracle.time_bucket(dts, div, nb))
+
+
+def _cfg(**kw):
+    base = dict(io_dtype=hstu.HSTU_DTYPE_BF16, compute_dtype=hstu.HSTU_DTYPE_BF16, n_norm=0,
+                pos_buckets=129, pos_clamp=128, time_buckets=128, time_log_div=0.301,
+                ln_eps=1e-5, max_tokens=1024, max_users=8)
+    d = kw.pop("d", 256)
+    H = kw.pop("H", 4)
+    base.update(kw)
+    return hstu.make_config(d, H, **base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=256, H=3), hstu.HSTU_ERR_INVALID_ARG),          # d != H * hd
+    (dict(d=256, H=8), hstu.HSTU_ERR_UNSUPPORTED),          # hd 32 on the tensor-core path
+    (dict(pos_clamp=129), hstu.HSTU_ERR_INVALID_ARG),       # clamp outside the table
+    (dict(time_buckets=0), hstu.HSTU_ERR_INVALID_ARG),
+    (dict(time_log_div=0.0), hstu.HSTU_ERR_INVALID_ARG),
+    (dict(max_tokens=2 ** 31), hstu.HSTU_ERR_INVALID_ARG),
+    (dict(io_dtype=7), hstu.HSTU_ERR_INVALID_ARG),
+    (dict(compute_dtype=hstu.HSTU_DTYPE_FP32), hstu.HSTU_ERR_UNSUPPORTED),  # fp32 math, bf16 io
+    (dict(d=320, H=5), hstu.HSTU_ERR_UNSUPPORTED),
+])
+def test_create_rejects_bad_configs_before_touching_cuda(lib, kw, status):
+    h = ctypes.c_void_p()
+    cfg = _cfg(**kw)
+    assert lib.hstu_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == status
+    assert not h.value
+
+
+def test_null_arguments_are_rejected(lib):
+    assert lib.hstu_create(None, 0, None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_destroy(None) == hstu.HSTU_OK
+    w = hstu.hstu_layer_weights()
+    assert lib.hstu_layer_forward(None, None, 0, None, 0, None, ctypes.byref(w), 0, None, None,
+                                  None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_get_device_error(None, None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_time_bucket_thresholds(0.301, 0, None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_debug_umma_tile(0, None, None, None, 128, 64) == hstu.HSTU_ERR_INVALID_ARG
