@@ -51,15 +51,23 @@ def oracle_inputs(batch, storage):
     return wl.round_to_storage(batch.x, storage).astype(np.float64)
 
 
-def teacher_forced_attention(uvqk_gpu, batch, cfg, params):
-    """The oracle's equation (2) evaluated on the GPU's own U,V,Q,K."""
+def teacher_forced_attention(uvqk_gpu, batch, cfg, params, with_abs=False):
+    """The oracle's equation (2) evaluated on the GPU's own U,V,Q,K.
+
+    With ``with_abs`` also returns sum_j |a_ij| |v_j| (the scale of the
+    rounding error of each output element)."""
     d = cfg.d_model
     V = uvqk_gpu[:, d:2 * d]
     Q = uvqk_gpu[:, 2 * d:3 * d]
     K = uvqk_gpu[:, 3 * d:]
-    return oracle.pointwise_attention(Q, K, V, batch.seq_offsets, batch.timestamps,
-                                      batch.num_candidates, params["rab_pos"], params["rab_time"],
-                                      cfg)
+    args = (batch.seq_offsets, batch.timestamps, batch.num_candidates, params["rab_pos"],
+            params["rab_time"], cfg)
+    O = oracle.pointwise_attention(Q, K, V, *args)
+    if not with_abs:
+        return O
+    O_abs = oracle.pointwise_attention(Q, K, np.abs(V), *args,
+                                       phi2=lambda s: np.abs(oracle.silu(s)))
+    return O, O_abs
 
 
 def rel_err(gpu, ref):

@@ -2,13 +2,17 @@
 
 Tolerances (inputs identical on both sides: the oracle receives the exact
 values stored in HBM):
-  fp32 path      Y max-abs <= 1e-4; intermediates <= 1e-5 x RMS (fp32 sums of
-                 <= 129 terms carry <= 129 * 2^-24 relative error)
-  bf16 path      Y max-abs <= 2e-2 x RMS(Y).  U,V,Q,K are stored in bf16:
-                 per element |err| <= 2^-8 |ref| + 1e-3 RMS.  The attention
-                 output O is compared with the oracle's equation (2) evaluated
-                 on the GPU's own U,V,Q,K (so only the kernel's own rounding
-                 remains: P in bf16, fp32 accumulation): <= 1e-2 x RMS.
+  fp32 path   Y max-abs <= 1e-4; intermediates <= 1e-5 x RMS (fp32 sums of
+              <= 129 terms carry <= 129 * 2^-24 relative error).
+  bf16 path   Y max-abs <= 2e-2 x RMS(Y).
+              U,V,Q,K and G are stored in bf16 (half an ulp is 2^-9 of the
+              value): per element |err| <= 2^-8 |ref| + 1e-3 RMS(ref).
+              The attention output O is compared with the oracle's equation
+              (2) evaluated on the GPU's own U,V,Q,K, so only the kernel's own
+              rounding remains (P in bf16, tanh-based SiLU within 2^-10,
+              fp32 accumulation): per element
+              |err| <= 2^-7 * sum_j |a_ij| |v_j| + 1e-6 RMS(O),
+              the standard bound of a dot product with relative term errors.
 Bucket indices and the mask are compared bit for bit.
 """
 import numpy as np
@@ -55,7 +59,7 @@ def test_umma_tile_layouts(mode, n, k):
 
 # ------------------------------------------------------------ workloads
 
-def _check_layer(w, batch, res, *, tf_tol=1e-2):
+def _check_layer(w, batch, res):
     cfg = cfg_for_workload(w)
     p = oracle_params(batch.layers[0], w.compute)
     X = oracle_inputs(batch, w.storage)
@@ -74,10 +78,13 @@ def _check_layer(w, batch, res, *, tf_tol=1e-2):
     uvqk = np.concatenate([ref["U"], ref["V"], ref["Q"], ref["K"]], axis=1)
     r = np.sqrt(np.mean(uvqk ** 2))
     assert np.all(np.abs(res["UVQK"] - uvqk) <= 2.0 ** -8 * np.abs(uvqk) + 1e-3 * r)
-    O_tf = teacher_forced_attention(res["UVQK"], batch, cfg, p)
-    assert rel_err(res["AV"], O_tf) <= tf_tol
+    O_tf, O_abs = teacher_forced_attention(res["UVQK"], batch, cfg, p, with_abs=True)
+    rO = np.sqrt(np.mean(O_tf ** 2)) if O_tf.size else 0.0
+    assert np.all(np.abs(res["AV"] - O_tf) <= 2.0 ** -7 * O_abs + 1e-6 * rO)
     N_tf = oracle.layer_norm(res["AV"], p["ln_gamma"], p["ln_beta"], cfg.ln_eps)
-    assert rel_err(res["G"], N_tf * res["UVQK"][:, :d]) <= 1e-2
+    G_tf = N_tf * res["UVQK"][:, :d]
+    rG = np.sqrt(np.mean(G_tf ** 2)) if G_tf.size else 0.0
+    assert np.all(np.abs(res["G"] - G_tf) <= 2.0 ** -8 * np.abs(G_tf) + 1e-3 * rG)
     return ref
 
 
