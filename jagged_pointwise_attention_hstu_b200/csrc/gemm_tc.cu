@@ -11,8 +11,9 @@
 //
 // Persistent, warp-specialised: warp 0 streams A/B k-blocks with TMA into a
 // 4-stage ring, warp 1 issues 128 x BN x 16 MMAs into one of two tensor-memory
-// accumulators, warps 2-5 drain the other accumulator through the fused
-// epilogue, so the epilogue of tile t overlaps the MMAs of tile t+1.
+// accumulators, warps 2-9 drain the other accumulator through the fused
+// epilogue (two warps per tensor-memory lane quarter, each taking half of the
+// columns), so the epilogue of tile t overlaps the MMAs of tile t+1.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -48,10 +49,15 @@ struct GemmLayout {
   static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
 };
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + __expf(-v)); }
+// SiLU(v) = v / (1 + e^-v) with the hardware exp2 and reciprocal (relative
+// error ~1e-7, far below the bf16 rounding that follows).  For v < -88 the
+// exponential overflows to +inf and the quotient is -0, the correct limit.
+__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
+
+constexpr int kGemmThreads = 320;
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
                    const __grid_constant__ CUtensorMap tma_b, const GemmParams p) {
   using L = GemmLayout<BN>;
@@ -76,7 +82,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], 256);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -156,9 +162,11 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // epilogue: warps 2..5, each owns the 32 tensor-memory lanes of its quarter
+    // epilogue: warps 2..9; warp w reads the 32 tensor-memory lanes of quarter
+    // w % 4 and the column half (w - 2) / 4 of the tile
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int c_begin = ((warp - 2) >> 2) * (BN / 2);
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
@@ -169,7 +177,7 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t grow = mt * 128 + row;
       const bool valid = grow < p.M;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = c_begin; c < c_begin + BN / 2; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + acc * BN + c + (uint32_t(q * 32) << 16), r);
         tmem_ld_wait();
@@ -270,7 +278,7 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   p.error = error;
   const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
   const int grid = int(tiles < num_sms ? tiles : num_sms);
-  gemm_tc_kernel<BN><<<grid, 192, L::kSmemBytes, st>>>(ta, tb, p);
+  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, p);
   return cudaGetLastError();
 }
 
