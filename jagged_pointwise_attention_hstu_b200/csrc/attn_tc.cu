@@ -7,17 +7,20 @@
 // (same blog, section "不对序列做 softmax"), hence no running maximum and no
 // rescaling of the accumulator, and the n x n score matrix is never stored.
 //
-// One CTA computes one (128-query tile, head) work item with 10 warps:
-//   warp 0      TMA: Q once, then K and V tiles into NS-stage rings
-//   warp 1      MMA issue: S_j = Q K_j^T into tensor-memory score buffer j % 2
+// One CTA computes one (128-query tile, head) work item with 12 warps:
+//   warp 0      TMA: Q once, then K tiles into an NSK-stage ring
+//   warp 1      MMA issue: S_j = Q K_j^T into tensor-memory score buffer j % 3
 //               (SS form, both operands K-major in shared memory), and
 //               O += P_j V_j with P_j read back from tensor memory (TS form,
 //               V consumed N-major straight from its row-major tile)
-//   warps 2-5   row group 0, one query row per thread, key tiles j = 0, 2, 4..
-//   warps 6-9   row group 1, same rows, key tiles j = 1, 3, 5..
+//   warp 2      TMA: V tiles and the keys' timestamps into an NSV-stage ring
+//   warps 4-7   row group 0, one query row per thread, key tiles j = 0, 2, 4..
+//   warps 8-11  row group 1, same rows, key tiles j = 1, 3, 5..
 // A row group reads S_j from tensor memory, adds the position and time
 // biases, applies the mask and SiLU and writes P_j (bf16) over the first half
-// of S_j's columns, while the tensor cores run S_{j+1} and P_{j-1} V_{j-1}.
+// of S_j's columns.  Three score buffers let the tensor cores run S_{j+1},
+// S_{j+2} and P_{j-1} V_{j-1} while the groups work on tiles j and j+1, and
+// separate K and V rings keep the key loads ahead of the value loads.
 //
 // Key tiles: only tiles that hold a visible key for some row of the query
 // tile are visited (see sched.cu); the last one is always the diagonal tile.
@@ -29,16 +32,21 @@
 // Each row keeps its current time bucket b and the key-timestamp cut
 // t_i - thr[b] (thr[k] = the smallest integer gap of bucket >= k, built on the
 // host from the fp64 rule), so an integer compare reproduces
-// floor(ln(1 + dt) / div) exactly.  Per (warp, key tile) the rows are
-// classified once:
+// floor(ln(1 + dt) / div) exactly.  The keys' timestamps arrive by TMA with
+// each V tile.  Per (warp, key tile) the rows are classified once:
 //   kFast  every key visible to every row of the warp and one time bucket per
 //          row: the whole bias is a per-row constant (plus the position
 //          gather when the position bucket is not clamped);
-//   kMed   every key visible, at most two time buckets per row: one 32-bit
-//          compare of the key's timestamp (relative to the tile's first key)
-//          against the row's cut picks the bias;
-//   kGen   anything else (diagonal tiles, user and history boundaries): the
-//          mask, the position clamp and the bucket walk per score.
+//   kMed   every key visible, at most two time buckets per row: one compare
+//          of the key's timestamp against the row's cut picks the bias;
+//   kAny   every key visible to every row, or history rows whose user starts
+//          at or before the tile (the causal diagonal), with gaps below 2^31:
+//          the exact bucket of each gap without a walk -- v = dt + 1, a table
+//          indexed by floor(log2 v) and the next two bits gives the bucket at
+//          the bin's low edge (a bin spans less than one bucket), and one
+//          compare against the next integer threshold corrects it;
+//   kGen   anything else (user and history boundaries, candidates): the full
+//          mask, position clamp and bucket walk per score.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -53,14 +61,16 @@ using namespace sm100;
 
 constexpr int kMaxPosEntries = 4097;   // pos_clamp <= 4096
 constexpr int kMaxTimeBuckets = 256;
-constexpr int kThreads = 320;
-constexpr int kFast = 0, kMed = 1, kGen = 2;
+constexpr int kThreads = 384;
+constexpr int kFast = 0, kMed = 1, kAny = 2, kGen = 3;
 
 struct AttnParams {
   const RowInfo* rows;
   const int32_t* order;
   const int64_t* ts;
   const int64_t* thresholds;
+  const uint8_t* time_lut;
+  const int32_t* thr32;
   const float* rab_pos;
   const float* rab_time;
   const int32_t* counters;
@@ -70,6 +80,7 @@ struct AttnParams {
   int d, H, num_qtiles;
   int pos_clamp, time_buckets;
   int n_norm_fixed;
+  int lut_exact;
   int32_t* dump_pidx;
   int32_t* dump_tidx;
   uint8_t* dump_vis;
@@ -77,18 +88,26 @@ struct AttnParams {
 
 template <int HD>
 struct AttnLayout {
-  static constexpr int NS = HD == 128 ? 2 : 3;
+  static constexpr int NSK = HD == 128 ? 3 : 4;   // K ring stages
+  static constexpr int NSV = HD == 128 ? 2 : 3;   // V ring stages
   static constexpr uint32_t kTileBytes = 128 * HD * 2;
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kTileBytes;
-  static constexpr uint32_t kV = kK + NS * kTileBytes;
-  static constexpr uint32_t kRabPos = kV + NS * kTileBytes;
+  static constexpr uint32_t kV = kK + NSK * kTileBytes;
+  static constexpr uint32_t kKts = kV + NSV * kTileBytes;            // int64 [stage][128], TMA
+  static constexpr uint32_t kRabPos = kKts + NSV * 128 * 8;
   static constexpr uint32_t kRabTime = kRabPos + ((kMaxPosEntries * 4 + 15) / 16) * 16;
   static constexpr uint32_t kThr = kRabTime + kMaxTimeBuckets * 4;
-  static constexpr uint32_t kKts = kThr + kMaxTimeBuckets * 8;       // int64 [group][buf][128]
-  static constexpr uint32_t kKrel = kKts + 2 * 2 * 128 * 8;          // int32 [group][buf][128]
-  static constexpr uint32_t kBars = kKrel + 2 * 2 * 128 * 4;
+  static constexpr uint32_t kThr32 = kThr + kMaxTimeBuckets * 8;     // int32 [257] (+pad)
+  static constexpr uint32_t kLut = kThr32 + 260 * 4;                 // uint8 [128]
+  static constexpr uint32_t kBars = kLut + 128;
   static constexpr uint32_t kSmemBytes = kBars + 256 + 1024;
+  // every TMA destination starts on a 1024-byte (swizzled tiles) or 128-byte boundary
+  static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "tile alignment");
+  static_assert(kTileBytes % 1024 == 0, "tile stride alignment");
+  static_assert(kKts % 128 == 0, "timestamp stage alignment");
+  static_assert(kBars % 8 == 0, "mbarrier alignment");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ int bucket_search(const int64_t* thr, int nb, int64_t dt) {
@@ -125,7 +144,7 @@ struct Row {
   int b, b_last;                        // time bucket at the walk position / tile end
   int64_t ti, cut, cut_last;
   float hc, hc_hi, hc_lo;               // half-bias constants of the fast paths
-  int cutr;                             // 32-bit cut relative to the tile's first key
+  uint32_t ti_lo;                       // low 32 bits of t_i (kAny)
 };
 
 struct Record {
@@ -136,104 +155,148 @@ struct Record {
   bool on;
 };
 
+// One score element: returns P (bf16-ready float) for key column jr of the tile.
+template <int MODE, bool PC, bool RECORD>
+__device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R,
+                                           const float* s_rp, const float* s_rt,
+                                           const int64_t* s_thr, const uint8_t* s_lut,
+                                           const int32_t* s_thr32, int clamp, const Record& rec) {
+  if constexpr (MODE == kFast || MODE == kMed) {
+    float add;
+    int tb = R.b;
+    if constexpr (MODE == kFast) {
+      add = R.hc;
+    } else {
+      const bool hi = tk <= R.cut;
+      add = hi ? R.hc_hi : R.hc_lo;
+      tb = hi ? R.b : R.b_last;
+    }
+    int pidx = clamp;
+    if constexpr (!PC) {
+      pidx = min(R.pos_rel - jr, clamp);
+      add = fmaf(0.5f, s_rp[pidx], add);
+    }
+    if constexpr (RECORD) {
+      if (rec.on) {
+        const int64_t at = rec.i * rec.T + rec.kb + jr;
+        rec.pidx[at] = pidx;
+        rec.tidx[at] = tb;
+        rec.vis[at] = 1;
+      }
+    }
+    return silu_half(fmaf(acc, 0.5f, add));
+  } else if constexpr (MODE == kAny) {
+    const bool vis = jr <= R.i_rel;
+    const uint32_t dd = R.ti_lo - uint32_t(tk);     // the gap; < 2^31 - 1 for visible keys
+    // masked keys may hold any gap (even -1, i.e. v = 0): keep v >= 1 so the
+    // table index stays in [0, 127] for every input
+    const uint32_t v = max(dd + 1u, 1u);
+    const int lz = __clz(int(v));
+    const int m = int(((v << lz) << 1) >> 30);
+    const int cand = s_lut[(((31 - lz) << 2) | m) & 127];
+    const int tb = cand + (int(dd) >= s_thr32[cand + 1] ? 1 : 0);
+    const int pidx = min(max(R.pos_rel - jr, 0), clamp);
+    if constexpr (RECORD) {
+      if (rec.on && rec.kb + jr < rec.T) {
+        const int64_t at = rec.i * rec.T + rec.kb + jr;
+        rec.pidx[at] = pidx;
+        rec.tidx[at] = tb;
+        rec.vis[at] = vis ? 1 : 0;
+      }
+    }
+    const float hh = 0.5f * (acc + s_rp[pidx] + s_rt[tb]);
+    return vis ? silu_half(hh) : 0.0f;
+  } else {
+    if (jr >= R.lo_rel && jr <= R.i_rel) walk_to(R.b, R.cut, tk, R.ti, s_thr);
+    const int dp = R.pos_rel - jr;
+    const int pidx = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+    const bool vis = (unsigned(jr - R.lo_rel) < unsigned(R.hi_rel - R.lo_rel)) || jr == R.i_rel;
+    if constexpr (RECORD) {
+      if (rec.on && rec.kb + jr < rec.T) {
+        const int64_t at = rec.i * rec.T + rec.kb + jr;
+        rec.pidx[at] = pidx;
+        rec.tidx[at] = R.b;
+        rec.vis[at] = vis ? 1 : 0;
+      }
+    }
+    const float sc = acc + s_rp[pidx] + s_rt[R.b];
+    return vis ? silu_half(0.5f * sc) : 0.0f;
+  }
+}
+
+template <int MODE, bool PC, bool RECORD>
+__device__ __forceinline__ void score_chunk(const uint32_t (&r)[16], int c, uint32_t taddr,
+                                            Row& R, const float* s_rp, const float* s_rt,
+                                            const int64_t* s_thr, const uint8_t* s_lut,
+                                            const int32_t* s_thr32, const int64_t* kts, int clamp,
+                                            const Record& rec) {
+  uint32_t pk[8];
+  const longlong2* k2 = reinterpret_cast<const longlong2*>(kts + c * 16);
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    int64_t t0 = 0, t1 = 0;
+    if constexpr (MODE != kFast) {
+      const longlong2 kk = k2[e >> 1];
+      t0 = kk.x;
+      t1 = kk.y;
+    }
+    const float p0 = score_one<MODE, PC, RECORD>(__uint_as_float(r[e]), c * 16 + e, t0, R, s_rp,
+                                                 s_rt, s_thr, s_lut, s_thr32, clamp, rec);
+    const float p1 = score_one<MODE, PC, RECORD>(__uint_as_float(r[e + 1]), c * 16 + e + 1, t1,
+                                                 R, s_rp, s_rt, s_thr, s_lut, s_thr32, clamp, rec);
+    pk[e >> 1] = pack_bf16x2(p0, p1);
+  }
+  tmem_st8(taddr + c * 8, pk);
+}
+
+// Scores one 128-key tile of S for this thread's row and writes P over its
+// first 64 columns, 16 keys at a time; the tensor-memory load of the next 16
+// scores overlaps the SiLU of the current ones.  P chunk c lands on columns
+// [8c, 8c + 8), which hold scores already consumed.
 template <int MODE, bool PC, bool RECORD>
 __device__ __forceinline__ void score_tile(uint32_t taddr, Row& R, const float* s_rp,
                                            const float* s_rt, const int64_t* s_thr,
-                                           const int64_t* kts, const int32_t* krel, int clamp,
-                                           const Record& rec) {
+                                           const uint8_t* s_lut, const int32_t* s_thr32,
+                                           const int64_t* kts, int clamp, const Record& rec) {
+  uint32_t ra[16], rb[16];
+  tmem_ld16(taddr, ra);
+  tmem_ld_wait();
 #pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
-    uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
+  for (int c = 0; c < 8; c += 2) {
+    tmem_ld16(taddr + (c + 1) * 16, rb);
+    score_chunk<MODE, PC, RECORD>(ra, c, taddr, R, s_rp, s_rt, s_thr, s_lut, s_thr32, kts, clamp, rec);
     tmem_ld_wait();
-    int kr[32];
-    if constexpr (MODE == kMed) {
-      const int4* k4 = reinterpret_cast<const int4*>(krel + c * 32);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int4 v = k4[q];
-        kr[4 * q + 0] = v.x; kr[4 * q + 1] = v.y; kr[4 * q + 2] = v.z; kr[4 * q + 3] = v.w;
-      }
-    }
-    uint32_t pk[16];
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      float pv[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int jr = c * 32 + e + u;
-        const float acc = __uint_as_float(r[e + u]);
-        if constexpr (MODE == kFast || MODE == kMed) {
-          float add;
-          int tb = R.b;
-          if constexpr (MODE == kFast) {
-            add = R.hc;
-          } else {
-            const bool hi = kr[e + u] <= R.cutr;
-            add = hi ? R.hc_hi : R.hc_lo;
-            tb = hi ? R.b : R.b_last;
-          }
-          int pidx = clamp;
-          if constexpr (!PC) {
-            pidx = min(R.pos_rel - jr, clamp);
-            add = fmaf(0.5f, s_rp[pidx], add);
-          }
-          pv[u] = silu_half(fmaf(acc, 0.5f, add));
-          if constexpr (RECORD) {
-            if (rec.on) {
-              const int64_t at = rec.i * rec.T + rec.kb + jr;
-              rec.pidx[at] = pidx;
-              rec.tidx[at] = tb;
-              rec.vis[at] = 1;
-            }
-          }
-        } else {
-          const int64_t tk = kts[jr];
-          if (jr >= R.lo_rel && jr <= R.i_rel) walk_to(R.b, R.cut, tk, R.ti, s_thr);
-          const int dp = R.pos_rel - jr;
-          const int pidx = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-          const bool vis = (unsigned(jr - R.lo_rel) < unsigned(R.hi_rel - R.lo_rel)) ||
-                           jr == R.i_rel;
-          const float sc = acc + s_rp[pidx] + s_rt[R.b];
-          pv[u] = vis ? silu_half(0.5f * sc) : 0.0f;
-          if constexpr (RECORD) {
-            if (rec.on && rec.kb + jr < rec.T) {
-              const int64_t at = rec.i * rec.T + rec.kb + jr;
-              rec.pidx[at] = pidx;
-              rec.tidx[at] = R.b;
-              rec.vis[at] = vis ? 1 : 0;
-            }
-          }
-        }
-      }
-      pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-    }
-    tmem_st16(taddr + c * 16, pk);
+    if (c + 2 < 8) tmem_ld16(taddr + (c + 2) * 16, ra);
+    score_chunk<MODE, PC, RECORD>(rb, c + 1, taddr, R, s_rp, s_rt, s_thr, s_lut, s_thr32, kts, clamp, rec);
+    tmem_ld_wait();
   }
 }
 
 template <int HD, bool RECORD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_ts,
+                   const AttnParams p) {
   using L = AttnLayout<HD>;
-  constexpr int NS = L::NS;
+  constexpr int NSK = L::NSK;
+  constexpr int NSV = L::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* s_rab_pos = reinterpret_cast<float*>(smem + L::kRabPos);
   float* s_rab_time = reinterpret_cast<float*>(smem + L::kRabTime);
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
+  int32_t* s_thr32 = reinterpret_cast<int32_t*>(smem + L::kThr32);
+  uint8_t* s_lut = reinterpret_cast<uint8_t*>(smem + L::kLut);
   int64_t* s_kts = reinterpret_cast<int64_t*>(smem + L::kKts);
-  int32_t* s_krel = reinterpret_cast<int32_t*>(smem + L::kKrel);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
-  uint64_t* k_empty = k_full + NS;
-  uint64_t* v_full = k_empty + NS;
-  uint64_t* v_empty = v_full + NS;
-  uint64_t* s_full = v_empty + NS;   // [2]
-  uint64_t* p_full = s_full + 2;     // [2]
-  uint64_t* o_full = p_full + 2;
+  uint64_t* k_empty = k_full + NSK;
+  uint64_t* v_full = k_empty + NSK;
+  uint64_t* v_empty = v_full + NSV;
+  uint64_t* s_full = v_empty + NSV;  // [3]
+  uint64_t* p_full = s_full + 3;     // [3]
+  uint64_t* o_full = p_full + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -257,13 +320,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 128);
     }
@@ -279,23 +344,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tS = tmem_base;          // two 128-column score buffers
-  const uint32_t tO = tmem_base + 256;    // HD-column output accumulator
+  const uint32_t tS = tmem_base;          // three 128-column score buffers
+  const uint32_t tO = tmem_base + 384;    // HD-column output accumulator
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ Q and K loads
     if (lane == 0) {
       prefetch_tmap(&tm);
       mbar_arrive_expect_tx(q_full, L::kTileBytes);
 #pragma unroll
       for (int b = 0; b < HD / 64; ++b)
         tma_load_2d(smem + L::kQ + b * 16384, &tm, q_full, 2 * d + h * HD + b * 64, int32_t(r0));
-      bool issued[NS];
-      uint32_t issued_ph[NS];
-      for (int s = 0; s < NS; ++s) issued[s] = false, issued_ph[s] = 0;
-      for (int j = 0; j < n_kt; ++j) {
-        const int s = j % NS;
-        const uint32_t ph = (j / NS) & 1;
+      bool issued[NSK];
+      uint32_t issued_ph[NSK];
+      for (int s = 0; s < NSK; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int s = j % NSK;
+        const uint32_t ph = (j / NSK) & 1;
         const int32_t key_row = int32_t((j < n_a ? kt_begin + j : qt)) * 128;
         if (!mbar_wait(&k_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
@@ -303,21 +368,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(smem + L::kK + s * L::kTileBytes + b * 16384, &tm, &k_full[s],
                       3 * d + h * HD + b * 64, key_row);
-        if (!mbar_wait(&v_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
-#pragma unroll
-        for (int b = 0; b < HD / 64; ++b)
-          tma_load_2d(smem + L::kV + s * L::kTileBytes + b * 16384, &tm, &v_full[s],
-                      d + h * HD + b * 64, key_row);
         issued[s] = true;
         issued_ph[s] = ph;
       }
       mbar_wait(q_full, 0);
-      for (int s = 0; s < NS; ++s)
-        if (issued[s]) {
-          mbar_wait(&k_full[s], issued_ph[s]);
-          mbar_wait(&v_full[s], issued_ph[s]);
-        }
+      for (int s = 0; s < NSK; ++s)
+        if (issued[s]) mbar_wait(&k_full[s], issued_ph[s]);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V + key timestamp loads
+    if (lane == 0) {
+      prefetch_tmap(&tm_ts);
+      bool issued[NSV];
+      uint32_t issued_ph[NSV];
+      for (int s = 0; s < NSV; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int s = j % NSV;
+        const uint32_t ph = (j / NSV) & 1;
+        const int32_t key_row = int32_t((j < n_a ? kt_begin + j : qt)) * 128;
+        if (!mbar_wait(&v_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes + 128 * 8);
+#pragma unroll
+        for (int b = 0; b < HD / 64; ++b)
+          tma_load_2d(smem + L::kV + s * L::kTileBytes + b * 16384, &tm, &v_full[s],
+                      d + h * HD + b * 64, key_row);
+        tma_load_1d(s_kts + s * 128, &tm_ts, &v_full[s], key_row);
+        issued[s] = true;
+        issued_ph[s] = ph;
+      }
+      for (int s = 0; s < NSV; ++s)
+        if (issued[s]) mbar_wait(&v_full[s], issued_ph[s]);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -328,31 +408,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0);
       tc_fence_after();
       auto issue_qk = [&](int j) -> bool {
-        const int s = j % NS;
-        if (!mbar_wait(&k_full[s], (j / NS) & 1)) return false;
+        const int s = j % NSK;
+        if (!mbar_wait(&k_full[s], (j / NSK) & 1)) return false;
         tc_fence_after();
         const uint32_t sK = smem_u32(smem + L::kK + s * L::kTileBytes);
-        const uint32_t dS = tS + (j & 1) * 128;
+        const uint32_t dS = tS + (j % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
           umma_ss(dS, desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024), idesc_qk,
                   kk > 0);
         }
-        umma_commit(&s_full[j & 1]);
+        umma_commit(&s_full[j % 3]);
         umma_commit(&k_empty[s]);
         return true;
       };
+      // QK runs two tiles ahead: S_{j+2} reuses the buffer of S_{j-1}, whose
+      // P_{j-1} V_{j-1} was issued (and executes in order) before it.
       if (ok) ok = issue_qk(0);
+      if (ok && n_kt > 1) ok = issue_qk(1);
       for (int j = 0; ok && j < n_kt; ++j) {
-        if (j + 1 < n_kt && !issue_qk(j + 1)) { ok = false; break; }
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+        if (j + 2 < n_kt && !issue_qk(j + 2)) { ok = false; break; }
+        if (!mbar_wait(&p_full[j % 3], (j / 3) & 1)) { ok = false; break; }
         tc_fence_after();
-        const int s = j % NS;
-        if (!mbar_wait(&v_full[s], (j / NS) & 1)) { ok = false; break; }
+        const int s = j % NSV;
+        if (!mbar_wait(&v_full[s], (j / NSV) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sV = smem_u32(smem + L::kV + s * L::kTileBytes);
-        const uint32_t aP = tS + (j & 1) * 128;
+        const uint32_t aP = tS + (j % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           umma_ts(tO, aP + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
@@ -364,40 +447,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(o_full);   // also drains: fires once every MMA above is done
       mbar_wait(o_full, 0);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ row groups
-    const int g = (warp - 2) >> 2;             // row group 0 or 1
-    const int t = threadIdx.x - 64 - 128 * g;  // 0..127 inside the group
+    const int g = (warp - 4) >> 2;             // row group 0 or 1
     const int q = warp & 3;                    // tensor-memory lane quarter
     const int row = q * 32 + lane;             // query row inside the tile
     const uint32_t lane_off = uint32_t(q * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
-    const int bar_id = 1 + g;
-    // tables: each group loads half, then both groups meet once
-    for (int k = threadIdx.x - 64; k <= clamp; k += 256) s_rab_pos[k] = p.rab_pos[k];
-    for (int k = threadIdx.x - 64; k < nb; k += 256) {
+    for (int k = threadIdx.x - 128; k <= clamp; k += 256) s_rab_pos[k] = p.rab_pos[k];
+    for (int k = threadIdx.x - 128; k < nb; k += 256) {
       s_rab_time[k] = p.rab_time[k];
       s_thr[k] = p.thresholds[k];
     }
-    int64_t* kts_g = s_kts + g * 256;
-    int32_t* krel_g = s_krel + g * 256;
-    auto key_base = [&](int j) -> int64_t { return int64_t(j < n_a ? kt_begin + j : qt) * 128; };
-    auto load_key = [&](int j, int64_t& tsv, int32_t& rel) {
-      const int64_t kb = key_base(j);
-      const int64_t t0 = p.ts[kb];
-      tsv = (kb + t < p.T) ? p.ts[kb + t] : t0;
-      const int64_t dr = tsv - t0;
-      rel = dr < 0 ? 0 : (dr > 0x7FFFFFFF ? 0x7FFFFFFF : int32_t(dr));
-    };
-    if (g < n_kt) {
-      int64_t tsv;
-      int32_t rel;
-      load_key(g, tsv, rel);
-      kts_g[t] = tsv;
-      krel_g[t] = rel;
-    }
-    named_bar_sync(3, 256);
+    for (int k = threadIdx.x - 128; k < 257; k += 256) s_thr32[k] = p.thr32[k];
+    if (threadIdx.x - 128 < 128) s_lut[threadIdx.x - 128] = p.time_lut[threadIdx.x - 128];
+    named_bar_sync(1, 256);
 
     const int64_t i = r0 + row;
     const bool valid = i < p.T;
@@ -411,6 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       pos = ri.pos;
       R.ti = p.ts[i];
     }
+    R.ti_lo = uint32_t(R.ti);
+    const bool history = valid && hi == i + 1 && pos == i;
     R.b = 0;
     R.cut = R.ti;
     if (valid) {
@@ -421,16 +488,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
     bool aborted = false;
 
-    int n = 0;
-    for (int j = g; j < n_kt; j += 2, ++n) {
-      const int buf = n & 1;
-      const int64_t kb = key_base(j);
-      int64_t nxt_ts = 0;
-      int32_t nxt_rel = 0;
-      if (j + 2 < n_kt) load_key(j + 2, nxt_ts, nxt_rel);
-      const int64_t* kts = kts_g + buf * 128;
-      const int32_t* krel = krel_g + buf * 128;
-
+    for (int j = g; j < n_kt; j += 2) {
+      const int64_t kb = int64_t(j < n_a ? kt_begin + j : qt) * 128;
+      const int s = j % NSV;
+      const int64_t* kts = s_kts + s * 128;
+      bool ok = aborted ? false : mbar_wait(&s_full[j % 3], (j / 3) & 1);
+      if (ok) ok = mbar_wait(&v_full[s], (j / NSV) & 1);   // key timestamps of tile j
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        aborted = true;
+        *abort_flag = 1;
+        continue;
+      }
       // ---- classify this row for the tile
       R.lo_rel = clamp_i32(lo - kb, -1, 129);
       R.hi_rel = clamp_i32(hi - kb, -1, 129);
@@ -446,18 +515,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk_to(R.b_last, R.cut_last, kts[127], R.ti, s_thr);
         lev = R.b - R.b_last;
       }
-      const bool wide = (kts[127] - kts[0]) >= int64_t(0x7FFFFFFE);
-      const int mode = __all_sync(0xffffffffu, full && lev == 0)
-                           ? kFast
-                           : (__all_sync(0xffffffffu, full && lev <= 1 && !wide) ? kMed : kGen);
+      int mode;
+      if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
+      else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
+      else if (p.lut_exact &&
+               __all_sync(0xffffffffu, (full || (history && lo <= kb)) &&
+                                           R.ti - kts[0] < int64_t(0x7FFFFFFE)))
+        mode = kAny;
+      else mode = kGen;
       const bool pc = __all_sync(0xffffffffu, posc);
-      if (mode != kGen) {
+      if (mode == kFast || mode == kMed) {
         const float rp_c = pc ? s_rab_pos[clamp] : 0.0f;
         R.hc_hi = 0.5f * (rp_c + s_rab_time[R.b]);
         R.hc_lo = 0.5f * (rp_c + s_rab_time[R.b_last]);
         R.hc = R.hc_hi;
-        const int64_t cr = R.cut - kts[0];
-        R.cutr = cr < -1 ? -1 : (cr > 0x7FFFFFFE ? 0x7FFFFFFE : int32_t(cr));
       }
       Record rec;
       rec.pidx = p.dump_pidx;
@@ -468,35 +539,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       rec.kb = kb;
       rec.on = RECORD && h == 0 && valid;
 
-      bool ok = aborted ? false : mbar_wait(&s_full[j & 1], (j >> 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        aborted = true;
-        *abort_flag = 1;
+      tc_fence_after();
+      const uint32_t taddr = tS + (j % 3) * 128 + lane_off;
+      if (mode == kFast) {
+        if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+      } else if (mode == kMed) {
+        if (pc) score_tile<kMed, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        else score_tile<kMed, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+      } else if (mode == kAny) {
+        score_tile<kAny, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+      } else {
+        score_tile<kGen, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
       }
-      if (!aborted) {
-        tc_fence_after();
-        const uint32_t taddr = tS + (j & 1) * 128 + lane_off;
-        if (mode == kFast) {
-          if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, kts, krel, clamp, rec);
-          else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, kts, krel, clamp, rec);
-        } else if (mode == kMed) {
-          if (pc) score_tile<kMed, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, kts, krel, clamp, rec);
-          else score_tile<kMed, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, kts, krel, clamp, rec);
-        } else {
-          score_tile<kGen, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, kts, krel, clamp, rec);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_full[j & 1]);
-      }
-      if (mode != kGen) {
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[j % 3]);
+      if (mode == kFast || mode == kMed) {
         R.b = R.b_last;
         R.cut = R.cut_last;
       }
-      kts_g[(buf ^ 1) * 128 + t] = nxt_ts;
-      krel_g[(buf ^ 1) * 128 + t] = nxt_rel;
-      named_bar_sync(bar_id, 128);
     }
 
     bool ok = aborted ? false : mbar_wait(o_full, 0);
@@ -536,10 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int HD, bool RECORD>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<HD>;
-  CUtensorMap tm;
+  CUtensorMap tm, tm_ts;
   if (!make_tmap_2d_bf16(&tm, a.uvqk, uint64_t(4 * a.d), uint64_t(a.T), uint64_t(4 * a.d) * 2,
                          64, 128))
     return cudaErrorInvalidValue;
+  if (!make_tmap_1d_i64(&tm_ts, a.ts, uint64_t(a.T), 128)) return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, RECORD>,
@@ -553,6 +616,9 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   p.order = a.order;
   p.ts = a.ts;
   p.thresholds = a.thresholds;
+  p.time_lut = a.time_lut;
+  p.thr32 = a.thr32;
+  p.lut_exact = a.lut_exact;
   p.rab_pos = a.rab_pos;
   p.rab_time = a.rab_time;
   p.counters = a.counters;
@@ -569,7 +635,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   p.dump_tidx = a.dump_tidx;
   p.dump_vis = a.dump_vis;
   const int64_t grid = int64_t(a.num_qtiles) * a.H;
-  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::kSmemBytes, st>>>(tm, p);
+  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::kSmemBytes, st>>>(tm, tm_ts, p);
   return cudaGetLastError();
 }
 

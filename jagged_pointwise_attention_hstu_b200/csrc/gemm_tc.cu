@@ -47,6 +47,8 @@ struct GemmLayout {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kBarOffset = kStages * kStageBytes;
   static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
+  static_assert(kABytes % 1024 == 0 && kStageBytes % 1024 == 0, "TMA destinations 1024-aligned");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 // SiLU(v) = v / (1 + e^-v) with the hardware exp2 and reciprocal (relative

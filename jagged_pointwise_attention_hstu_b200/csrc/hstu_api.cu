@@ -38,6 +38,31 @@ int64_t fp64_bucket(int64_t dt, double div) {
   return static_cast<int64_t>(floor(log(1.0 + static_cast<double>(dt)) / div));
 }
 
+// Candidate-bucket table for 32-bit gaps: bin (e, m) holds v = dt + 1 with
+// floor(log2 v) = e and the two bits after the leading one equal to m, so a
+// bin spans at most a factor 1.25 in v (0.223 in ln v), less than one bucket
+// (0.301 for the layer's divisor; the table is only used when div > 0.223).
+// The bucket of any gap in a bin is therefore the bin's low-edge bucket or the
+// next one, and one compare against the next threshold decides.
+void build_time_lut(const int64_t* thr, int nb, uint8_t* lut, int32_t* thr32) {
+  for (int e = 0; e < 32; ++e)
+    for (int m = 0; m < 4; ++m) {
+      int64_t vlow;
+      if (e == 0) vlow = 1;
+      else if (e == 1) vlow = m < 2 ? 2 : 3;
+      else vlow = (int64_t(1) << e) + int64_t(m) * (int64_t(1) << (e - 2));
+      const int64_t dt = vlow - 1;
+      int b = 0;
+      for (int k = 1; k < nb; ++k)
+        if (dt >= thr[k]) b = k;
+      lut[e * 4 + m] = uint8_t(b);
+    }
+  for (int k = 0; k < 257; ++k) {
+    const int64_t t = k < nb ? thr[k] : int64_t(0x7FFFFFFF);
+    thr32[k] = t > 0x7FFFFFFF ? 0x7FFFFFFF : int32_t(t);
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <typename T>
@@ -61,6 +86,18 @@ bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_1d_i64(CUtensorMap* m, const void* base, uint64_t n, uint32_t box) {
+  auto fn = encode_fn();
+  if (fn == nullptr || n == 0) return false;
+  cuuint64_t dims[1] = {n};
+  cuuint64_t strides[1] = {n * 8};
+  cuuint32_t boxd[1] = {box};
+  cuuint32_t estr[1] = {1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_INT64, 1, const_cast<void*>(base), dims, strides, boxd,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace hstu
@@ -135,6 +172,7 @@ hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** ou
     delete h;
     return HSTU_ERR_INVALID_ARG;
   }
+  hstu::build_time_lut(h->thresholds_host, c.time_buckets, h->time_lut_host, h->thr32_host);
   const size_t T = size_t(c.max_tokens);
   const size_t cs = hstu::elem_size(c.compute_dtype);
   const size_t nqt = (T + hstu::kTile - 1) / hstu::kTile + 1;
@@ -151,6 +189,10 @@ hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** ou
   if (e == cudaSuccess) e = hstu::alloc(&ws.counters, 16);
   if (e == cudaSuccess) e = hstu::alloc(&ws.error, 16);
   if (e == cudaSuccess) e = hstu::alloc(&ws.thresholds, 256 * 8);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.time_lut, 128);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.thr32, 257 * 4);
+  if (e == cudaSuccess) e = cudaMemcpy(ws.time_lut, h->time_lut_host, 128, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(ws.thr32, h->thr32_host, 257 * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(ws.error, 0, 16);
   if (e == cudaSuccess)
     e = cudaMemcpy(ws.thresholds, h->thresholds_host, size_t(c.time_buckets) * 8,
@@ -170,7 +212,7 @@ hstu_status hstu_destroy(hstu_handle* h) {
   cudaDeviceSynchronize();
   Workspace& ws = h->ws;
   void* ptrs[] = {ws.xb, ws.uvqk, ws.av, ws.g, ws.rows, ws.qtile_order, ws.qtile_cost,
-                  ws.counters, ws.error, ws.thresholds};
+                  ws.counters, ws.error, ws.thresholds, ws.time_lut, ws.thr32};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   if (h->timer.created)
@@ -245,6 +287,9 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   a.order = ws.qtile_order;
   a.ts = ts;
   a.thresholds = ws.thresholds;
+  a.time_lut = ws.time_lut;
+  a.thr32 = ws.thr32;
+  a.lut_exact = c.time_log_div > 0.2232 ? 1 : 0;
   a.rab_pos = w->rab_pos;
   a.rab_time = w->rab_time;
   a.counters = ws.counters;
@@ -430,6 +475,9 @@ hstu_status hstu_debug_attention_buckets(hstu_handle* h, int64_t T, const int32_
   a.order = h->ws.qtile_order;
   a.ts = ts;
   a.thresholds = h->ws.thresholds;
+  a.time_lut = h->ws.time_lut;
+  a.thr32 = h->ws.thr32;
+  a.lut_exact = c.time_log_div > 0.2232 ? 1 : 0;
   a.rab_pos = zeros;
   a.rab_time = zeros + c.pos_buckets;
   a.counters = h->ws.counters;

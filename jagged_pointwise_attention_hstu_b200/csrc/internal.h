@@ -32,6 +32,8 @@ struct Workspace {
   int32_t* counters = nullptr;     // [4]: n_norm, max cost, scratch
   int32_t* error = nullptr;        // device error word
   int64_t* thresholds = nullptr;   // [time_buckets] time-bucket thresholds
+  uint8_t* time_lut = nullptr;     // [128] bucket at the low edge of each log2 quarter-octave bin
+  int32_t* thr32 = nullptr;        // [257] thresholds capped to int32, padded with INT32_MAX
 };
 
 }  // namespace hstu
@@ -56,6 +58,8 @@ struct hstu_handle_s {
   hstu::Workspace ws;
   int64_t last_T = 0;
   int64_t thresholds_host[256];
+  uint8_t time_lut_host[128];
+  int32_t thr32_host[257];
 };
 
 namespace hstu {
@@ -91,6 +95,8 @@ struct AttnArgs {
   const int32_t* order;      // q-tile order
   const int64_t* ts;
   const int64_t* thresholds; // [time_buckets]
+  const uint8_t* time_lut;   // [128]
+  const int32_t* thr32;      // [257]
   const float* rab_pos;
   const float* rab_time;
   const int32_t* counters;   // [0] = n_norm
@@ -100,6 +106,7 @@ struct AttnArgs {
   int pos_clamp, time_buckets;
   int n_norm_fixed;          // > 0: use it; else counters[0]
   int num_qtiles;
+  int lut_exact;             // time_log_div > ln 1.25: the candidate-bucket table is exact
   // recording variant
   int32_t* dump_pidx;
   int32_t* dump_tidx;
@@ -124,5 +131,6 @@ cudaError_t run_umma_tile(int mode, const void* a, const void* b, float* c, int 
 // tensor maps (hstu_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_1d_i64(CUtensorMap* m, const void* base, uint64_t n, uint32_t box);
 
 }  // namespace hstu
