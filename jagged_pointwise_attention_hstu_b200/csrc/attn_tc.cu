@@ -7,20 +7,22 @@
 // (same blog, section "不对序列做 softmax"), hence no running maximum and no
 // rescaling of the accumulator, and the n x n score matrix is never stored.
 //
-// One CTA computes one (128-query tile, head) work item with 12 warps:
-//   warp 0      TMA: Q once, then K tiles into an NSK-stage ring
-//   warp 1      MMA issue: S_j = Q K_j^T into tensor-memory score buffer j % 3
-//               (SS form, both operands K-major in shared memory), and
-//               O += P_j V_j with P_j read back from tensor memory (TS form,
+// One CTA computes one work item -- a pair of adjacent 128-query tiles and
+// one head -- with 12 warps:
+//   warp 0      TMA: both Q tiles once, then K tiles into an NSK-stage ring
+//   warp 1      MMA issue: S_q = Q_q K_j^T into tensor-memory score buffer q
+//               (SS form, both operands K-major in shared memory) and
+//               O_q += P_q V_j with P_q read back from tensor memory (TS form,
 //               V consumed N-major straight from its row-major tile)
 //   warp 2      TMA: V tiles and the keys' timestamps into an NSV-stage ring
-//   warps 4-7   row group 0, one query row per thread, key tiles j = 0, 2, 4..
-//   warps 8-11  row group 1, same rows, key tiles j = 1, 3, 5..
-// A row group reads S_j from tensor memory, adds the position and time
-// biases, applies the mask and SiLU and writes P_j (bf16) over the first half
-// of S_j's columns.  Three score buffers let the tensor cores run S_{j+1},
-// S_{j+2} and P_{j-1} V_{j-1} while the groups work on tiles j and j+1, and
-// separate K and V rings keep the key loads ahead of the value loads.
+//   warps 4-7   row group 0: one row of query tile 0 per thread
+//   warps 8-11  row group 1: one row of query tile 1 per thread
+// A row group reads S_q from tensor memory, adds the position and time
+// biases, applies the mask and SiLU and writes P_q (bf16) over the first half
+// of S_q's columns.  The MMAs ping-pong between the query tiles -- while group
+// 0 scores key tile j, the tensor cores run S_1 = Q_1 K_j^T and P_0 V_{j-1} --
+// and every K and V tile loaded feeds both query tiles, which halves the K/V
+// traffic per flop.
 //
 // Key tiles: only tiles that hold a visible key for some row of the query
 // tile are visited (see sched.cu); the last one is always the diagonal tile.
@@ -62,7 +64,7 @@ using namespace sm100;
 constexpr int kMaxPosEntries = 4097;   // pos_clamp <= 4096
 constexpr int kMaxTimeBuckets = 256;
 constexpr int kThreads = 384;
-constexpr int kFast = 0, kMed = 1, kAny = 2, kGen = 3;
+constexpr int kFast = 0, kMed = 1, kAny = 2, kGen = 3, kZero = 4;
 
 struct AttnParams {
   const RowInfo* rows;
@@ -77,7 +79,7 @@ struct AttnParams {
   int32_t* error;
   float* av;
   int64_t T;
-  int d, H, num_qtiles;
+  int d, H, num_pairs;
   int pos_clamp, time_buckets;
   int n_norm_fixed;
   int lut_exact;
@@ -88,26 +90,28 @@ struct AttnParams {
 
 template <int HD>
 struct AttnLayout {
-  static constexpr int NSK = HD == 128 ? 3 : 4;   // K ring stages
+  static constexpr int NSK = HD == 128 ? 2 : 3;   // K ring stages
   static constexpr int NSV = HD == 128 ? 2 : 3;   // V ring stages
   static constexpr uint32_t kTileBytes = 128 * HD * 2;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTileBytes;
+  static constexpr uint32_t kQ = 0;                                  // two Q tiles
+  static constexpr uint32_t kK = kQ + 2 * kTileBytes;
   static constexpr uint32_t kV = kK + NSK * kTileBytes;
   static constexpr uint32_t kKts = kV + NSV * kTileBytes;            // int64 [stage][128], TMA
-  static constexpr uint32_t kRabPos = kKts + NSV * 128 * 8;
-  static constexpr uint32_t kRabTime = kRabPos + ((kMaxPosEntries * 4 + 15) / 16) * 16;
-  static constexpr uint32_t kThr = kRabTime + kMaxTimeBuckets * 4;
+  static constexpr uint32_t kThr = kKts + NSV * 128 * 8;
   static constexpr uint32_t kThr32 = kThr + kMaxTimeBuckets * 8;     // int32 [257] (+pad)
   static constexpr uint32_t kLut = kThr32 + 260 * 4;                 // uint8 [128]
-  static constexpr uint32_t kBars = kLut + 128;
-  static constexpr uint32_t kSmemBytes = kBars + 256 + 1024;
+  static constexpr uint32_t kRabTime = kLut + 128;
+  static constexpr uint32_t kBars = kRabTime + kMaxTimeBuckets * 4;
+  static constexpr uint32_t kRabPos = kBars + 256;                   // float [clamp + 1]
+  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
+    return kRabPos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16 + 1024;
+  }
   // every TMA destination starts on a 1024-byte (swizzled tiles) or 128-byte boundary
   static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "tile alignment");
   static_assert(kTileBytes % 1024 == 0, "tile stride alignment");
   static_assert(kKts % 128 == 0, "timestamp stage alignment");
   static_assert(kBars % 8 == 0, "mbarrier alignment");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ int bucket_search(const int64_t* thr, int nb, int64_t dt) {
@@ -249,20 +253,65 @@ __device__ __forceinline__ void score_chunk(const uint32_t (&r)[16], int c, uint
   tmem_st8(taddr + c * 8, pk);
 }
 
+// Writes P = 0 for a tile whose keys are all later than every row of the warp.
+template <bool RECORD>
+__device__ __forceinline__ void zero_tile(uint32_t taddr, const Record& rec) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) pk[e] = 0u;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) tmem_st8(taddr + c * 8, pk);
+  if constexpr (RECORD) {
+    if (rec.on)
+      for (int jr = 0; jr < 128 && rec.kb + jr < rec.T; ++jr) {
+        const int64_t at = rec.i * rec.T + rec.kb + jr;
+        rec.pidx[at] = 0;
+        rec.tidx[at] = 0;
+        rec.vis[at] = 0;
+      }
+  }
+}
+
 // Scores one 128-key tile of S for this thread's row and writes P over its
 // first 64 columns, 16 keys at a time; the tensor-memory load of the next 16
 // scores overlaps the SiLU of the current ones.  P chunk c lands on columns
-// [8c, 8c + 8), which hold scores already consumed.
+// [8c, 8c + 8), which hold scores already consumed.  On the masked paths a
+// chunk whose keys are all later than every row of the warp is written as 0
+// without being scored.
 template <int MODE, bool PC, bool RECORD>
 __device__ __forceinline__ void score_tile(uint32_t taddr, Row& R, const float* s_rp,
                                            const float* s_rt, const int64_t* s_thr,
                                            const uint8_t* s_lut, const int32_t* s_thr32,
                                            const int64_t* kts, int clamp, const Record& rec) {
+  int live = 8;   // chunks holding a key visible to some row of the warp
+  if constexpr (MODE == kAny || MODE == kGen) {
+    int last = R.i_rel;   // every visible key of the row is <= its own column
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    live = min(8, last / 16 + 1);
+  }
   uint32_t ra[16], rb[16];
   tmem_ld16(taddr, ra);
   tmem_ld_wait();
 #pragma unroll 1
   for (int c = 0; c < 8; c += 2) {
+    if (c >= live) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pk[e] = 0u;
+      tmem_st8(taddr + c * 8, pk);
+      tmem_st8(taddr + (c + 1) * 8, pk);
+      if constexpr (RECORD) {
+        if (rec.on)
+          for (int jr = c * 16; jr < 128 && rec.kb + jr < rec.T; ++jr) {
+            const int64_t at = rec.i * rec.T + rec.kb + jr;
+            rec.pidx[at] = 0;
+            rec.tidx[at] = 0;
+            rec.vis[at] = 0;
+          }
+      }
+      continue;
+    }
     tmem_ld16(taddr + (c + 1) * 16, rb);
     score_chunk<MODE, PC, RECORD>(ra, c, taddr, R, s_rp, s_rt, s_thr, s_lut, s_thr32, kts, clamp, rec);
     tmem_ld_wait();
@@ -294,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_empty = k_full + NSK;
   uint64_t* v_full = k_empty + NSK;
   uint64_t* v_empty = v_full + NSV;
-  uint64_t* s_full = v_empty + NSV;  // [3]
-  uint64_t* p_full = s_full + 3;     // [3]
-  uint64_t* o_full = p_full + 3;
+  uint64_t* s_full = v_empty + NSV;  // [2] one per query tile
+  uint64_t* p_full = s_full + 2;     // [2]
+  uint64_t* o_full = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -304,19 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int d = p.d;
 
-  // ---- work item (head-major) and its key-tile range
+  // ---- work item (head-major) and its key tiles
   const int w = blockIdx.x;
-  const int h = w / p.num_qtiles;
-  const int qt = p.order[w % p.num_qtiles];
-  const int64_t r0 = int64_t(qt) * 128;
-  const RowInfo ri0 = p.rows[r0];
-  int64_t lo0 = ri0.lo;
-  if (lo0 < 0 || lo0 > r0) lo0 = r0;
-  int64_t vis_end = ri0.hi < r0 ? int64_t(ri0.hi) : r0;
-  if (vis_end < lo0) vis_end = lo0;
-  const int kt_begin = int(lo0 / 128);
-  const int n_a = int((vis_end + 127) / 128) - kt_begin;   // tiles before the diagonal
-  const int n_kt = n_a + 1;
+  const int h = w / p.num_pairs;
+  const int pr = p.order[w % p.num_pairs];
+  const int qt0 = 2 * pr;
+  const PairTiles pt = pair_tiles(p.rows, p.T, pr);
+  const int nq = pt.n_diag;              // query tiles in this pair (1 or 2)
+  const int n_a = pt.n_a;
+  const int n_kt = n_a + nq;
+  auto key_tile = [&](int j) -> int { return j < n_a ? pt.a_lo + j : qt0 + (j - n_a); };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -328,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 128);
     }
@@ -344,30 +390,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tS = tmem_base;          // three 128-column score buffers
-  const uint32_t tO = tmem_base + 384;    // HD-column output accumulator
+  // columns: S_0 [0,128), S_1 [128,256), O_0 [256, 256+HD), O_1 [256+HD, 256+2HD)
+  auto tS = [&](int q) -> uint32_t { return tmem_base + q * 128; };
+  auto tO = [&](int q) -> uint32_t { return tmem_base + 256 + q * HD; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ Q and K loads
     if (lane == 0) {
       prefetch_tmap(&tm);
-      mbar_arrive_expect_tx(q_full, L::kTileBytes);
+      mbar_arrive_expect_tx(q_full, nq * L::kTileBytes);
+      for (int q = 0; q < nq; ++q)
 #pragma unroll
-      for (int b = 0; b < HD / 64; ++b)
-        tma_load_2d(smem + L::kQ + b * 16384, &tm, q_full, 2 * d + h * HD + b * 64, int32_t(r0));
+        for (int b = 0; b < HD / 64; ++b)
+          tma_load_2d(smem + L::kQ + q * L::kTileBytes + b * 16384, &tm, q_full,
+                      2 * d + h * HD + b * 64, (qt0 + q) * 128);
       bool issued[NSK];
       uint32_t issued_ph[NSK];
       for (int s = 0; s < NSK; ++s) issued[s] = false, issued_ph[s] = 0;
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int s = j % NSK;
         const uint32_t ph = (j / NSK) & 1;
-        const int32_t key_row = int32_t((j < n_a ? kt_begin + j : qt)) * 128;
         if (!mbar_wait(&k_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(smem + L::kK + s * L::kTileBytes + b * 16384, &tm, &k_full[s],
-                      3 * d + h * HD + b * 64, key_row);
+                      3 * d + h * HD + b * 64, key_tile(j) * 128);
         issued[s] = true;
         issued_ph[s] = ph;
       }
@@ -385,14 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int s = j % NSV;
         const uint32_t ph = (j / NSV) & 1;
-        const int32_t key_row = int32_t((j < n_a ? kt_begin + j : qt)) * 128;
         if (!mbar_wait(&v_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&v_full[s], L::kTileBytes + 128 * 8);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(smem + L::kV + s * L::kTileBytes + b * 16384, &tm, &v_full[s],
-                      d + h * HD + b * 64, key_row);
-        tma_load_1d(s_kts + s * 128, &tm_ts, &v_full[s], key_row);
+                      d + h * HD + b * 64, key_tile(j) * 128);
+        tma_load_1d(s_kts + s * 128, &tm_ts, &v_full[s], key_tile(j) * 128);
         issued[s] = true;
         issued_ph[s] = ph;
       }
@@ -404,44 +451,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, HD, false, true);
-      const uint32_t sQ = smem_u32(smem + L::kQ);
       bool ok = mbar_wait(q_full, 0);
       tc_fence_after();
-      auto issue_qk = [&](int j) -> bool {
+      // S_q = Q_q K_j^T; after the last query tile of key tile j the K stage is released
+      auto issue_qk = [&](int q, int j) -> bool {
         const int s = j % NSK;
         if (!mbar_wait(&k_full[s], (j / NSK) & 1)) return false;
         tc_fence_after();
+        const uint32_t sQ = smem_u32(smem + L::kQ + q * L::kTileBytes);
         const uint32_t sK = smem_u32(smem + L::kK + s * L::kTileBytes);
-        const uint32_t dS = tS + (j % 3) * 128;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(dS, desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024), idesc_qk,
-                  kk > 0);
+          umma_ss(tS(q), desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024),
+                  idesc_qk, kk > 0);
         }
-        umma_commit(&s_full[j % 3]);
-        umma_commit(&k_empty[s]);
+        umma_commit(&s_full[q]);
+        if (q == nq - 1) umma_commit(&k_empty[s]);
         return true;
       };
-      // QK runs two tiles ahead: S_{j+2} reuses the buffer of S_{j-1}, whose
-      // P_{j-1} V_{j-1} was issued (and executes in order) before it.
-      if (ok) ok = issue_qk(0);
-      if (ok && n_kt > 1) ok = issue_qk(1);
+      for (int q = 0; ok && q < nq; ++q) ok = issue_qk(q, 0);
       for (int j = 0; ok && j < n_kt; ++j) {
-        if (j + 2 < n_kt && !issue_qk(j + 2)) { ok = false; break; }
-        if (!mbar_wait(&p_full[j % 3], (j / 3) & 1)) { ok = false; break; }
-        tc_fence_after();
         const int s = j % NSV;
         if (!mbar_wait(&v_full[s], (j / NSV) & 1)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t sV = smem_u32(smem + L::kV + s * L::kTileBytes);
-        const uint32_t aP = tS + (j % 3) * 128;
+        for (int q = 0; ok && q < nq; ++q) {
+          if (!mbar_wait(&p_full[q], j & 1)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_ts(tO, aP + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
-                  (j > 0 || kk > 0));
+          for (int kk = 0; kk < 8; ++kk) {
+            umma_ts(tO(q), tS(q) + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
+                    (j > 0 || kk > 0));
+          }
+          if (q == nq - 1) umma_commit(&v_empty[s]);
+          // S_q is rewritten only after P_q V_j (issued just above, executed in order)
+          if (j + 1 < n_kt && !issue_qk(q, j + 1)) ok = false;
         }
-        umma_commit(&v_empty[s]);
       }
       if (!ok) *abort_flag = 1;
       umma_commit(o_full);   // also drains: fires once every MMA above is done
@@ -449,10 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ row groups
-    const int g = (warp - 4) >> 2;             // row group 0 or 1
-    const int q = warp & 3;                    // tensor-memory lane quarter
-    const int row = q * 32 + lane;             // query row inside the tile
-    const uint32_t lane_off = uint32_t(q * 32) << 16;
+    const int q = (warp - 4) >> 2;             // query tile of this row group
+    const int wq = warp & 3;                   // tensor-memory lane quarter
+    const int row = wq * 32 + lane;            // query row inside the tile
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
     for (int k = threadIdx.x - 128; k <= clamp; k += 256) s_rab_pos[k] = p.rab_pos[k];
@@ -464,8 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x - 128 < 128) s_lut[threadIdx.x - 128] = p.time_lut[threadIdx.x - 128];
     named_bar_sync(1, 256);
 
-    const int64_t i = r0 + row;
-    const bool valid = i < p.T;
+    const int64_t i = int64_t(qt0 + q) * 128 + row;
+    const bool valid = q < nq && i < p.T;
     int64_t lo = 0, hi = 0, pos = 0;   // rows past T see nothing
     Row R;
     R.ti = 0;
@@ -488,11 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
     bool aborted = false;
 
-    for (int j = g; j < n_kt; j += 2) {
-      const int64_t kb = int64_t(j < n_a ? kt_begin + j : qt) * 128;
+    for (int j = 0; q < nq && j < n_kt; ++j) {
+      const int64_t kb = int64_t(key_tile(j)) * 128;
       const int s = j % NSV;
       const int64_t* kts = s_kts + s * 128;
-      bool ok = aborted ? false : mbar_wait(&s_full[j % 3], (j / 3) & 1);
+      bool ok = aborted ? false : mbar_wait(&s_full[q], j & 1);
       if (ok) ok = mbar_wait(&v_full[s], (j / NSV) & 1);   // key timestamps of tile j
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -516,7 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         lev = R.b - R.b_last;
       }
       int mode;
-      if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
+      if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
+      else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
       else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
       else if (p.lut_exact &&
                __all_sync(0xffffffffu, (full || (history && lo <= kb)) &&
@@ -540,8 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       rec.on = RECORD && h == 0 && valid;
 
       tc_fence_after();
-      const uint32_t taddr = tS + (j % 3) * 128 + lane_off;
-      if (mode == kFast) {
+      const uint32_t taddr = tS(q) + lane_off;
+      if (mode == kZero) {
+        zero_tile<RECORD>(taddr, rec);
+      } else if (mode == kFast) {
         if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
         else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
       } else if (mode == kMed) {
@@ -554,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[j % 3]);
+      mbar_arrive(&p_full[q]);
       if (mode == kFast || mode == kMed) {
         R.b = R.b_last;
         R.cut = R.cut_last;
@@ -563,13 +611,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool ok = aborted ? false : mbar_wait(o_full, 0);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    if (ok && q < nq) {
       tc_fence_after();
-      // group g writes the columns [g * HD / 2, (g + 1) * HD / 2) of its rows
 #pragma unroll 1
-      for (int c = g * (HD / 64); c < (g + 1) * (HD / 64); ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tO + lane_off + c * 32, r);
+        tmem_ld32(tO(q) + lane_off + c * 32, r);
         tmem_ld_wait();
         if (valid) {
           float4* dst = reinterpret_cast<float4*>(p.av + i * d + h * HD + c * 32);
@@ -581,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(r[4 * e + 3]) * inv_nn);
         }
       }
-    } else {
+    } else if (!ok) {
       *abort_flag = 1;
     }
   }
@@ -607,7 +654,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, RECORD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(L::kSmemBytes));
+                                         int(L::smem_bytes(kMaxPosEntries - 1)));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
@@ -627,15 +674,15 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   p.T = a.T;
   p.d = a.d;
   p.H = a.H;
-  p.num_qtiles = a.num_qtiles;
+  p.num_pairs = a.num_pairs;
   p.pos_clamp = a.pos_clamp;
   p.time_buckets = a.time_buckets;
   p.n_norm_fixed = a.n_norm_fixed;
   p.dump_pidx = a.dump_pidx;
   p.dump_tidx = a.dump_tidx;
   p.dump_vis = a.dump_vis;
-  const int64_t grid = int64_t(a.num_qtiles) * a.H;
-  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::kSmemBytes, st>>>(tm, tm_ts, p);
+  const int64_t grid = int64_t(a.num_pairs) * a.H;
+  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::smem_bytes(a.pos_clamp), st>>>(tm, tm_ts, p);
   return cudaGetLastError();
 }
 

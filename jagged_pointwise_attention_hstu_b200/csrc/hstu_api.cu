@@ -301,7 +301,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   a.pos_clamp = c.pos_clamp;
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
-  a.num_qtiles = int((T + hstu::kTile - 1) / hstu::kTile);
+  a.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
   if (f32) {
     {
       Timed tm(h, kF1, st);
@@ -489,7 +489,7 @@ hstu_status hstu_debug_attention_buckets(hstu_handle* h, int64_t T, const int32_
   a.pos_clamp = c.pos_clamp;
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
-  a.num_qtiles = int((T + hstu::kTile - 1) / hstu::kTile);
+  a.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
   a.dump_pidx = pidx_out;
   a.dump_tidx = tidx_out;
   a.dump_vis = vis_out;

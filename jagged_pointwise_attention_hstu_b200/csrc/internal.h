@@ -21,14 +21,57 @@ struct RowInfo {
   int32_t lo, hi, pos, user;
 };
 
+// Key tiles visited by the pair of query tiles (2p, 2p+1): the run
+// [a_lo, a_lo + n_a) of tiles before query tile 2p, then the diagonal tiles
+// 2p and, when it exists, 2p+1.  Every key visible to a row of either query
+// tile lies in these tiles: a query tile's earlier keys belong to the user of
+// its first row (users starting inside the tile see only the tile itself),
+// and a candidate sees only its history and itself.
+struct PairTiles {
+  int a_lo, n_a, n_diag;
+};
+
+__device__ __forceinline__ void range_before(const RowInfo* rows, int64_t r, int& a, int& e) {
+  const RowInfo ri = rows[r];
+  int64_t lo = ri.lo;
+  if (lo < 0 || lo > r) lo = r;
+  int64_t ve = ri.hi < r ? int64_t(ri.hi) : r;
+  if (ve < lo) ve = lo;
+  a = int(lo / kTile);
+  e = int((ve + kTile - 1) / kTile);
+}
+
+__device__ __forceinline__ PairTiles pair_tiles(const RowInfo* rows, int64_t T, int pr) {
+  const int qt0 = 2 * pr;
+  const int64_t r0 = int64_t(qt0) * kTile;
+  const int64_t r1 = r0 + kTile;
+  int a0, e0;
+  range_before(rows, r0, a0, e0);
+  PairTiles t;
+  t.n_diag = 1;
+  int a_lo = a0, a_hi = e0;
+  if (r1 < T) {
+    int a1, e1;
+    range_before(rows, r1, a1, e1);
+    a_lo = a1 < a0 ? a1 : a0;
+    a_hi = e1 > e0 ? e1 : e0;
+    t.n_diag = 2;
+  }
+  if (a_hi > qt0) a_hi = qt0;
+  if (a_hi < a_lo) a_hi = a_lo;
+  t.a_lo = a_lo;
+  t.n_a = a_hi - a_lo;
+  return t;
+}
+
 struct Workspace {
   void* xb = nullptr;          // [T, d] bf16: X cast for the GEMM when io is fp32
   void* uvqk = nullptr;        // [T, 4d] compute dtype
   float* av = nullptr;         // [T, d] fp32
   void* g = nullptr;           // [T, d] compute dtype
   RowInfo* rows = nullptr;     // [T]
-  int32_t* qtile_order = nullptr;  // [ceil(T / 128)] q-tiles by descending cost
-  int32_t* qtile_cost = nullptr;   // [ceil(T / 128)]
+  int32_t* qtile_order = nullptr;  // [ceil(T / 256)] q-tile pairs by descending cost
+  int32_t* qtile_cost = nullptr;   // [ceil(T / 256)]
   int32_t* counters = nullptr;     // [4]: n_norm, max cost, scratch
   int32_t* error = nullptr;        // device error word
   int64_t* thresholds = nullptr;   // [time_buckets] time-bucket thresholds
@@ -92,7 +135,7 @@ struct AttnArgs {
   const void* uvqk;          // [T, 4d] bf16
   float* av;                 // [T, d] fp32
   const RowInfo* rows;
-  const int32_t* order;      // q-tile order
+  const int32_t* order;      // q-tile pair order
   const int64_t* ts;
   const int64_t* thresholds; // [time_buckets]
   const uint8_t* time_lut;   // [128]
@@ -105,7 +148,7 @@ struct AttnArgs {
   int d, H, hd;
   int pos_clamp, time_buckets;
   int n_norm_fixed;          // > 0: use it; else counters[0]
-  int num_qtiles;
+  int num_pairs;             // ceil(T / 256)
   int lut_exact;             // time_log_div > ln 1.25: the candidate-bucket table is exact
   // recording variant
   int32_t* dump_pidx;

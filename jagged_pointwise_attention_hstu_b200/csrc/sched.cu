@@ -77,8 +77,9 @@ __global__ void rows_kernel(const int32_t* __restrict__ offs, int32_t B, int64_t
   if (bad) atomicOr(err, HSTU_DEVERR_TIMESTAMPS);
 }
 
-// One block: cost of every q-tile, then a counting sort by descending cost.
-__global__ void order_kernel(const RowInfo* __restrict__ rows, int64_t T, int32_t nqt,
+// One block: cost of every pair of query tiles (key tiles it visits), then a
+// counting sort by descending cost (longest processing time first).
+__global__ void order_kernel(const RowInfo* __restrict__ rows, int64_t T, int32_t npairs,
                              int32_t* __restrict__ cost, int32_t* __restrict__ order,
                              int32_t* __restrict__ counters) {
   constexpr int NB = 4096;   // cost bins; costs above NB-1 share the top bin
@@ -88,17 +89,10 @@ __global__ void order_kernel(const RowInfo* __restrict__ rows, int64_t T, int32_
   if (threadIdx.x == 0) s_max = 0;
   __syncthreads();
   int32_t local_max = 0;
-  for (int32_t qt = threadIdx.x; qt < nqt; qt += blockDim.x) {
-    const int64_t r0 = int64_t(qt) * kTile;
-    const RowInfo ri = rows[r0];
-    int64_t lo = ri.lo;
-    if (lo < 0 || lo > r0) lo = r0;
-    int64_t vis_end = ri.hi < r0 ? int64_t(ri.hi) : r0;
-    if (vis_end < lo) vis_end = lo;
-    const int32_t kt_begin = int32_t(lo / kTile);
-    const int32_t kt_end = int32_t((vis_end + kTile - 1) / kTile);
-    const int32_t c = (kt_end - kt_begin) + 1;
-    cost[qt] = c;
+  for (int32_t pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+    const PairTiles t = pair_tiles(rows, T, pr);
+    const int32_t c = t.n_a + t.n_diag;
+    cost[pr] = c;
     local_max = c > local_max ? c : local_max;
     atomicAdd(&hist[c < NB ? c : NB - 1], 1);
   }
@@ -115,10 +109,10 @@ __global__ void order_kernel(const RowInfo* __restrict__ rows, int64_t T, int32_
     counters[1] = s_max;
   }
   __syncthreads();
-  for (int32_t qt = threadIdx.x; qt < nqt; qt += blockDim.x) {
-    const int32_t c = cost[qt];
+  for (int32_t pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+    const int32_t c = cost[pr];
     const int32_t slot = atomicAdd(&hist[c < NB ? c : NB - 1], 1);
-    order[slot] = qt;
+    order[slot] = pr;
   }
 }
 
@@ -148,8 +142,8 @@ cudaError_t launch_schedule(const hstu_handle_s* h, int64_t T, const int32_t* of
                                           ts, ws.rows, ws.counters, ws.error);
   e = cudaGetLastError();
   if (e != cudaSuccess || T == 0) return e;
-  const int32_t nqt = int32_t((T + kTile - 1) / kTile);
-  order_kernel<<<1, 1024, 0, st>>>(ws.rows, T, nqt, ws.qtile_cost, ws.qtile_order, ws.counters);
+  const int32_t npairs = int32_t((T + 2 * kTile - 1) / (2 * kTile));
+  order_kernel<<<1, 1024, 0, st>>>(ws.rows, T, npairs, ws.qtile_cost, ws.qtile_order, ws.counters);
   return cudaGetLastError();
 }
 
