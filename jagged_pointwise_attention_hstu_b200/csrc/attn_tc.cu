@@ -39,14 +39,17 @@
 //   kFast  every key visible to every row of the warp and one time bucket per
 //          row: the whole bias is a per-row constant (plus the position
 //          gather when the position bucket is not clamped);
-//   kMed   every key visible, at most two time buckets per row: one compare
-//          of the key's timestamp against the row's cut picks the bias;
+//   kMed   every key visible, at most two time buckets per row: one 32-bit
+//          compare of the gap against the row's threshold picks the bias;
+//   kCut   every key visible, at most four time buckets per row: three such
+//          compares and a select chain;
 //   kAny   every key visible to every row, or history rows whose user starts
 //          at or before the tile (the causal diagonal), with gaps below 2^31:
-//          the exact bucket of each gap without a walk -- v = dt + 1, a table
-//          indexed by floor(log2 v) and the next two bits gives the bucket at
-//          the bin's low edge (a bin spans less than one bucket), and one
-//          compare against the next integer threshold corrects it;
+//          the exact bucket of each gap without a walk -- v = dt + 1 falls in a
+//          bin (floor(log2 v) and the next two bits) spanning less than one
+//          bucket; a per-CTA table gives, per bin, the next bucket's integer
+//          threshold and both candidate biases, so one 16-byte shared load
+//          and one compare give the time bias;
 //   kGen   anything else (user and history boundaries, candidates): the full
 //          mask, position clamp and bucket walk per score.
 #include <cuda.h>
@@ -64,7 +67,7 @@ using namespace sm100;
 constexpr int kMaxPosEntries = 4097;   // pos_clamp <= 4096
 constexpr int kMaxTimeBuckets = 256;
 constexpr int kThreads = 384;
-constexpr int kFast = 0, kMed = 1, kAny = 2, kGen = 3, kZero = 4;
+constexpr int kFast = 0, kMed = 1, kCut = 2, kAny = 3, kGen = 4, kZero = 5;
 
 struct AttnParams {
   const RowInfo* rows;
@@ -100,7 +103,8 @@ struct AttnLayout {
   static constexpr uint32_t kThr = kKts + NSV * 128 * 8;
   static constexpr uint32_t kThr32 = kThr + kMaxTimeBuckets * 8;     // int32 [257] (+pad)
   static constexpr uint32_t kLut = kThr32 + 260 * 4;                 // uint8 [128]
-  static constexpr uint32_t kRabTime = kLut + 128;
+  static constexpr uint32_t kAnyTab = kLut + 128;                    // int4 [128]
+  static constexpr uint32_t kRabTime = kAnyTab + 128 * 16;
   static constexpr uint32_t kBars = kRabTime + kMaxTimeBuckets * 4;
   static constexpr uint32_t kRabPos = kBars + 256;                   // float [clamp + 1]
   static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
@@ -148,7 +152,9 @@ struct Row {
   int b, b_last;                        // time bucket at the walk position / tile end
   int64_t ti, cut, cut_last;
   float hc, hc_hi, hc_lo;               // half-bias constants of the fast paths
-  uint32_t ti_lo;                       // low 32 bits of t_i (kAny)
+  float hc2, hc3;                       // kCut: half-bias of buckets b - 2, b - 3
+  int th1, th2, th3;                    // kMed/kCut: a gap below th_m drops a bucket
+  uint32_t ti_lo;                       // low 32 bits of t_i (kMed, kCut, kAny)
 };
 
 struct Record {
@@ -165,15 +171,20 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
                                            const float* s_rp, const float* s_rt,
                                            const int64_t* s_thr, const uint8_t* s_lut,
                                            const int32_t* s_thr32, int clamp, const Record& rec) {
-  if constexpr (MODE == kFast || MODE == kMed) {
-    float add;
+  if constexpr (MODE == kFast || MODE == kMed || MODE == kCut) {
+    float add = R.hc;
     int tb = R.b;
-    if constexpr (MODE == kFast) {
-      add = R.hc;
-    } else {
-      const bool hi = tk <= R.cut;
-      add = hi ? R.hc_hi : R.hc_lo;
-      tb = hi ? R.b : R.b_last;
+    if constexpr (MODE != kFast) {
+      const int dd = int(R.ti_lo - uint32_t(tk));   // the gap; in [0, 2^31) on these paths
+      const bool d1 = dd < R.th1;
+      add = d1 ? R.hc_lo : R.hc;
+      if constexpr (RECORD) tb = R.b - (d1 ? 1 : 0);
+      if constexpr (MODE == kCut) {
+        const bool d2 = dd < R.th2;
+        const bool d3 = dd < R.th3;
+        add = d2 ? (d3 ? R.hc3 : R.hc2) : add;
+        if constexpr (RECORD) tb -= (d2 ? 1 : 0) + (d3 ? 1 : 0);
+      }
     }
     int pidx = clamp;
     if constexpr (!PC) {
@@ -196,19 +207,20 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
     // table index stays in [0, 127] for every input
     const uint32_t v = max(dd + 1u, 1u);
     const int lz = __clz(int(v));
-    const int m = int(((v << lz) << 1) >> 30);
-    const int cand = s_lut[(((31 - lz) << 2) | m) & 127];
-    const int tb = cand + (int(dd) >= s_thr32[cand + 1] ? 1 : 0);
+    const int idx = (((31 - lz) << 2) | int((v << lz) >> 29 & 3u)) & 127;
+    const int4 ent = reinterpret_cast<const int4*>(s_lut)[idx];   // {thr, rt_lo, rt_hi, cand}
+    const bool up = int(dd) >= ent.x;
+    const float rt = __int_as_float(up ? ent.z : ent.y);
     const int pidx = min(max(R.pos_rel - jr, 0), clamp);
     if constexpr (RECORD) {
       if (rec.on && rec.kb + jr < rec.T) {
         const int64_t at = rec.i * rec.T + rec.kb + jr;
         rec.pidx[at] = pidx;
-        rec.tidx[at] = tb;
+        rec.tidx[at] = ent.w + (up ? 1 : 0);
         rec.vis[at] = vis ? 1 : 0;
       }
     }
-    const float hh = 0.5f * (acc + s_rp[pidx] + s_rt[tb]);
+    const float hh = 0.5f * (acc + s_rp[pidx] + rt);
     return vis ? silu_half(hh) : 0.0f;
   } else {
     if (jr >= R.lo_rel && jr <= R.i_rel) walk_to(R.b, R.cut, tk, R.ti, s_thr);
@@ -336,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
   int32_t* s_thr32 = reinterpret_cast<int32_t*>(smem + L::kThr32);
   uint8_t* s_lut = reinterpret_cast<uint8_t*>(smem + L::kLut);
+  int4* s_any = reinterpret_cast<int4*>(smem + L::kAnyTab);
   int64_t* s_kts = reinterpret_cast<int64_t*>(smem + L::kKts);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars;
@@ -508,6 +521,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = threadIdx.x - 128; k < 257; k += 256) s_thr32[k] = p.thr32[k];
     if (threadIdx.x - 128 < 128) s_lut[threadIdx.x - 128] = p.time_lut[threadIdx.x - 128];
     named_bar_sync(1, 256);
+    if (threadIdx.x - 128 < 128) {
+      // per bin: {threshold of the next bucket, bias of the bin's bucket, bias of the next, bucket}
+      const int idx = threadIdx.x - 128;
+      const int cand = s_lut[idx];
+      const int nxt = cand + 1 < nb ? cand + 1 : cand;
+      s_any[idx] = make_int4(cand + 1 < nb ? s_thr32[cand + 1] : 0x7FFFFFFF,
+                             __float_as_int(s_rab_time[cand]), __float_as_int(s_rab_time[nxt]),
+                             cand);
+    }
+    named_bar_sync(1, 256);
+    const uint8_t* s_anyb = reinterpret_cast<const uint8_t*>(s_any);
 
     const int64_t i = int64_t(qt0 + q) * 128 + row;
     const bool valid = q < nq && i < p.T;
@@ -560,21 +584,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk_to(R.b_last, R.cut_last, kts[127], R.ti, s_thr);
         lev = R.b - R.b_last;
       }
+      const bool narrow = R.ti - kts[0] < int64_t(0x7FFFFFFE);   // gaps fit in int32
       int mode;
       if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
       else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
-      else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
+      else if (__all_sync(0xffffffffu, full && lev <= 1 && narrow)) mode = kMed;
+      else if (__all_sync(0xffffffffu, full && lev <= 3 && narrow)) mode = kCut;
       else if (p.lut_exact &&
-               __all_sync(0xffffffffu, (full || (history && lo <= kb)) &&
-                                           R.ti - kts[0] < int64_t(0x7FFFFFFE)))
+               __all_sync(0xffffffffu, (full || (history && lo <= kb)) && narrow))
         mode = kAny;
       else mode = kGen;
       const bool pc = __all_sync(0xffffffffu, posc);
-      if (mode == kFast || mode == kMed) {
+      if (mode == kFast || mode == kMed || mode == kCut) {
+        // R.b = bucket of the tile's first key (the largest gap); a gap below
+        // thr[R.b - m + 1] drops the bucket below R.b - m + 1
         const float rp_c = pc ? s_rab_pos[clamp] : 0.0f;
-        R.hc_hi = 0.5f * (rp_c + s_rab_time[R.b]);
-        R.hc_lo = 0.5f * (rp_c + s_rab_time[R.b_last]);
-        R.hc = R.hc_hi;
+        const int b0 = R.b;
+        R.hc = 0.5f * (rp_c + s_rab_time[b0]);
+        R.hc_lo = 0.5f * (rp_c + s_rab_time[max(b0 - 1, 0)]);
+        R.hc2 = 0.5f * (rp_c + s_rab_time[max(b0 - 2, 0)]);
+        R.hc3 = 0.5f * (rp_c + s_rab_time[max(b0 - 3, 0)]);
+        R.th1 = s_thr32[b0];
+        R.th2 = s_thr32[max(b0 - 1, 0)];
+        R.th3 = s_thr32[max(b0 - 2, 0)];
       }
       Record rec;
       rec.pidx = p.dump_pidx;
@@ -590,20 +622,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mode == kZero) {
         zero_tile<RECORD>(taddr, rec);
       } else if (mode == kFast) {
-        if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
-        else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else if (mode == kMed) {
-        if (pc) score_tile<kMed, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
-        else score_tile<kMed, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        if (pc) score_tile<kMed, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kMed, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+      } else if (mode == kCut) {
+        if (pc) score_tile<kCut, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kCut, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else if (mode == kAny) {
-        score_tile<kAny, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        score_tile<kAny, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else {
-        score_tile<kGen, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_lut, s_thr32, kts, clamp, rec);
+        score_tile<kGen, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[q]);
-      if (mode == kFast || mode == kMed) {
+      if (mode == kFast || mode == kMed || mode == kCut) {
         R.b = R.b_last;
         R.cut = R.cut_last;
       }
