@@ -561,8 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t kb = int64_t(key_tile(j)) * 128;
       const int s = j % NSV;
       const int64_t* kts = s_kts + s * 128;
-      bool ok = aborted ? false : mbar_wait(&s_full[q], j & 1);
-      if (ok) ok = mbar_wait(&v_full[s], (j / NSV) & 1);   // key timestamps of tile j
+      // The key timestamps of tile j arrive with V_j, usually well before
+      // S_q(j) is ready: classify the rows first, off the critical path.
+      bool ok = aborted ? false : mbar_wait(&v_full[s], (j / NSV) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         aborted = true;
@@ -617,6 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       rec.kb = kb;
       rec.on = RECORD && h == 0 && valid;
 
+      ok = mbar_wait(&s_full[q], j & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        aborted = true;
+        *abort_flag = 1;
+        continue;
+      }
       tc_fence_after();
       const uint32_t taddr = tS(q) + lane_off;
       if (mode == kZero) {
