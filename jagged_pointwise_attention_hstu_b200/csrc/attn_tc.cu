@@ -99,8 +99,9 @@ struct AttnLayout {
   static constexpr uint32_t kQ = 0;                                  // two Q tiles
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;
   static constexpr uint32_t kV = kK + NSK * kTileBytes;
+  static constexpr int NST = 4;                   // key-timestamp ring stages
   static constexpr uint32_t kKts = kV + NSV * kTileBytes;            // int64 [stage][128], TMA
-  static constexpr uint32_t kThr = kKts + NSV * 128 * 8;
+  static constexpr uint32_t kThr = kKts + NST * 128 * 8;
   static constexpr uint32_t kThr32 = kThr + kMaxTimeBuckets * 8;     // int32 [257] (+pad)
   static constexpr uint32_t kLut = kThr32 + 260 * 4;                 // uint8 [128]
   static constexpr uint32_t kAnyTab = kLut + 128;                    // int4 [128]
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = AttnLayout<HD>;
   constexpr int NSK = L::NSK;
   constexpr int NSV = L::NSV;
+  constexpr int NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -359,7 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + NSV;  // [2] one per query tile
   uint64_t* p_full = s_full + 2;     // [2]
   uint64_t* o_full = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  uint64_t* t_full = o_full + 1;     // [NST] key timestamps of a tile landed
+  uint64_t* t_empty = t_full + NST;  // [NST] every row-group warp is done with them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + NST);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -392,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[b], 128);
     }
     mbar_init(o_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&t_full[s], 1);
+      mbar_init(&t_empty[s], 4 * nq);   // the warps of every row group that has rows
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -439,7 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ V + key timestamp loads
     if (lane == 0) {
-      prefetch_tmap(&tm_ts);
       bool issued[NSV];
       uint32_t issued_ph[NSV];
       for (int s = 0; s < NSV; ++s) issued[s] = false, issued_ph[s] = 0;
@@ -447,17 +454,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j % NSV;
         const uint32_t ph = (j / NSV) & 1;
         if (!mbar_wait(&v_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes + 128 * 8);
+        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(smem + L::kV + s * L::kTileBytes + b * 16384, &tm, &v_full[s],
                       d + h * HD + b * 64, key_tile(j) * 128);
-        tma_load_1d(s_kts + s * 128, &tm_ts, &v_full[s], key_tile(j) * 128);
         issued[s] = true;
         issued_ph[s] = ph;
       }
       for (int s = 0; s < NSV; ++s)
         if (issued[s]) mbar_wait(&v_full[s], issued_ph[s]);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ key timestamp loads
+    if (lane == 0) {
+      prefetch_tmap(&tm_ts);
+      bool issued[NST];
+      uint32_t issued_ph[NST];
+      for (int s = 0; s < NST; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int s = j % NST;
+        const uint32_t ph = (j / NST) & 1;
+        if (!mbar_wait(&t_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&t_full[s], 128 * 8);
+        tma_load_1d(s_kts + s * 128, &tm_ts, &t_full[s], key_tile(j) * 128);
+        issued[s] = true;
+        issued_ph[s] = ph;
+      }
+      for (int s = 0; s < NST; ++s)
+        if (issued[s]) mbar_wait(&t_full[s], issued_ph[s]);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -559,11 +584,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int j = 0; q < nq && j < n_kt; ++j) {
       const int64_t kb = int64_t(key_tile(j)) * 128;
-      const int s = j % NSV;
-      const int64_t* kts = s_kts + s * 128;
-      // The key timestamps of tile j arrive with V_j, usually well before
-      // S_q(j) is ready: classify the rows first, off the critical path.
-      bool ok = aborted ? false : mbar_wait(&v_full[s], (j / NSV) & 1);
+      const int st = j % NST;
+      const int64_t* kts = s_kts + st * 128;
+      // The key timestamps of tile j come through their own ring, loaded well
+      // ahead of the scores: classify the rows first, off the critical path.
+      bool ok = aborted ? false : mbar_wait(&t_full[st], (j / NST) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         aborted = true;
@@ -646,6 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[q]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[st]);
       if (mode == kFast || mode == kMed || mode == kCut) {
         R.b = R.b_last;
         R.cut = R.cut_last;
