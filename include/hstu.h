@@ -176,6 +176,51 @@ hstu_status hstu_set_kernel_timing(hstu_handle* h, int32_t enabled);
  * number of launches (host int64 [HSTU_KERNEL_KINDS]).  Either pointer may be NULL. */
 hstu_status hstu_get_kernel_timing(hstu_handle* h, double* total_ms, int64_t* launches);
 
+/* ---- Attention without allocation ----
+ * The pages have no counterpart of this entry point: it is an interface of
+ * this library for callers that may not allocate at call time.  It runs the
+ * attention step of equation (2) alone -- the scheduler and the fused
+ * tensor-core attention kernel of the BF16 path, the same kernels that
+ * hstu_layer_forward launches -- with every piece of scratch (per-token row
+ * facts, pair order and cost, counters, the error word, the time-bucket
+ * tables) in one fixed file-scope device array of this library, about 1 MiB
+ * per device, instead of a handle's workspace.  Neither the call nor anything
+ * it calls allocates host or device memory.
+ *   cfg            host; uses d_model, num_heads, head_dim, n_norm, pos_buckets,
+ *                  pos_clamp, time_buckets and time_log_div; compute_dtype must be
+ *                  BF16 and head_dim 64 or 128 (else HSTU_ERR_UNSUPPORTED);
+ *                  io_dtype, ln_eps, max_tokens and max_users are ignored
+ *   uvqk           device bf16 [T, 4d]: SiLU(X W1^T + b1), columns U | V | Q | K
+ *                  (only V, Q and K are read)
+ *   total_tokens   T, 0 <= T <= HSTU_NOALLOC_MAX_TOKENS; larger T returns
+ *                  HSTU_ERR_WORKSPACE before any launch
+ *   seq_offsets, num_users, timestamps, mask_mode, num_candidates
+ *                  as for hstu_layer_forward
+ *   rab_pos        device fp32 [pos_buckets]
+ *   rab_time       device fp32 [time_buckets]
+ *   av             device fp32 [T, d]: O of equation (2), divided by n_norm
+ *   device_error   device int32 or NULL: overwritten with this call's
+ *                  HSTU_DEVERR_* bits (0 = none), in stream order
+ *   stream         cudaStream_t or NULL
+ * Set-up: the first call on a device looks up the address of the scratch
+ * array there (cudaGetSymbolAddress, checked; HSTU_ERR_CUDA on failure) and
+ * caches it; make that first call outside any stream capture.  The bucket
+ * tables are rebuilt on the host when time_log_div or time_buckets changes.
+ * Every call first clears the scratch that must start at zero (the counters
+ * and the error word) and rewrites the tables, in stream order.
+ * The scratch is one per device and process: two calls on one device whose
+ * executions overlap (different streams, different host threads) race on it
+ * and give undefined results, so serialise them.  The host-side caches are
+ * not thread-safe either.  Calls are asynchronous on `stream`. */
+#define HSTU_NOALLOC_MAX_TOKENS 65536
+
+hstu_status hstu_attention_noalloc(const hstu_config* cfg, const void* uvqk, int64_t total_tokens,
+                                   const int32_t* seq_offsets, int32_t num_users,
+                                   const int64_t* timestamps, hstu_mask_mode mask_mode,
+                                   const int32_t* num_candidates, const float* rab_pos,
+                                   const float* rab_time, float* av, int32_t* device_error,
+                                   void* stream);
+
 /* ---- Inspection entry points for tests (same library, same kernels) ---- */
 
 typedef enum {

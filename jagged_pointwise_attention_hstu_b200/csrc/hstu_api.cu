@@ -545,3 +545,145 @@ hstu_status hstu_debug_umma_tile(int32_t mode, const void* a, const void* b, flo
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Attention without allocation.  Every piece of scratch of the attention step
+// (row facts, pair order and cost, counters, error word, bucket tables) lives
+// in one file-scope device array; the call allocates nothing.
+namespace hstu {
+namespace {
+
+constexpr int64_t kNoAllocMaxTokens = HSTU_NOALLOC_MAX_TOKENS;
+constexpr size_t kNoAllocPairs = 1024;   // >= kNoAllocMaxTokens / (2 * kTile)
+constexpr size_t kOffRows = 0;
+constexpr size_t kOffOrder = kOffRows + size_t(kNoAllocMaxTokens) * sizeof(RowInfo);
+constexpr size_t kOffCost = kOffOrder + kNoAllocPairs * 4;
+constexpr size_t kOffCounters = kOffCost + kNoAllocPairs * 4;
+constexpr size_t kOffError = kOffCounters + 256;
+constexpr size_t kOffThr = kOffError + 256;
+constexpr size_t kOffLut = kOffThr + 256 * 8;
+constexpr size_t kOffThr32 = kOffLut + 256;
+constexpr size_t kNoAllocScratchBytes = kOffThr32 + 1280;   // 1,060,864 bytes
+static_assert(kNoAllocPairs * 2 * kTile >= size_t(kNoAllocMaxTokens), "pair table size");
+static_assert(kOffOrder % 256 == 0 && kOffThr % 256 == 0 && kOffThr32 % 256 == 0, "alignment");
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Host cache of the scratch address per device (set on the first call on that device).
+constexpr int kNoAllocMaxDevices = 64;
+uint8_t* g_noalloc_addr[kNoAllocMaxDevices] = {nullptr};
+
+// Host cache of the bucket tables for the last (divisor, bucket count).
+struct NoAllocTables {
+  int64_t thr[256];
+  int32_t thr32[260];
+  uint8_t lut[128];
+  int32_t nb;
+};
+NoAllocTables g_noalloc_tables;
+double g_noalloc_div = 0.0;
+int32_t g_noalloc_nb = 0;
+
+// Writes the bucket tables (passed by value) into the scratch and clears the
+// counters and the error word: the scratch values that must start at zero.
+__global__ void noalloc_prepare_kernel(const NoAllocTables t, int64_t* thr, uint8_t* lut,
+                                       int32_t* thr32, int32_t* counters, int32_t* err) {
+  for (int k = threadIdx.x; k < 257; k += blockDim.x) {
+    thr32[k] = t.thr32[k];
+    if (k < t.nb) thr[k] = t.thr[k];
+    if (k < 128) lut[k] = t.lut[k];
+    if (k < 4) {
+      counters[k] = 0;
+      err[k] = 0;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" hstu_status hstu_attention_noalloc(const hstu_config* cfg, const void* uvqk,
+                                              int64_t T, const int32_t* offsets, int32_t B,
+                                              const int64_t* ts, hstu_mask_mode mode,
+                                              const int32_t* ncand, const float* rab_pos,
+                                              const float* rab_time, float* av,
+                                              int32_t* device_error, void* stream) {
+  using namespace hstu;
+  if (cfg == nullptr) return HSTU_ERR_INVALID_ARG;
+  const hstu_config& c = *cfg;
+  if (c.num_heads <= 0 || c.d_model != c.num_heads * c.head_dim) return HSTU_ERR_INVALID_ARG;
+  if (c.pos_buckets < 1 || c.pos_clamp < 0 || c.pos_clamp >= c.pos_buckets) return HSTU_ERR_INVALID_ARG;
+  if (c.time_buckets < 1 || c.time_buckets > 256 || !(c.time_log_div > 0.0)) return HSTU_ERR_INVALID_ARG;
+  if (c.compute_dtype != HSTU_DTYPE_BF16 || (c.head_dim != 64 && c.head_dim != 128) ||
+      c.d_model % 128 != 0 || c.d_model > 1024 || c.pos_clamp > 4096)
+    return HSTU_ERR_UNSUPPORTED;
+  if (T < 0 || B < 0 || (B == 0 && T != 0) || offsets == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (mode != HSTU_MASK_CAUSAL && mode != HSTU_MASK_MFALCON) return HSTU_ERR_INVALID_ARG;
+  if (mode == HSTU_MASK_MFALCON && B > 0 && ncand == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (T > kNoAllocMaxTokens) return HSTU_ERR_WORKSPACE;
+  if (T > 0) {
+    const void* ps[] = {uvqk, ts, av, rab_pos, rab_time};
+    for (const void* p : ps)
+      if (p == nullptr || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return HSTU_ERR_UNSUPPORTED;
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return HSTU_ERR_CUDA;
+    g_noalloc_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  if (g_noalloc_nb != c.time_buckets || g_noalloc_div != c.time_log_div) {
+    if (hstu_time_bucket_thresholds(c.time_log_div, c.time_buckets, g_noalloc_tables.thr) != HSTU_OK)
+      return HSTU_ERR_INVALID_ARG;
+    build_time_lut(g_noalloc_tables.thr, c.time_buckets, g_noalloc_tables.lut,
+                   g_noalloc_tables.thr32);
+    g_noalloc_tables.nb = c.time_buckets;
+    g_noalloc_nb = c.time_buckets;
+    g_noalloc_div = c.time_log_div;
+  }
+  uint8_t* base = g_noalloc_addr[dev];
+  RowInfo* rows = reinterpret_cast<RowInfo*>(base + kOffRows);
+  int32_t* order = reinterpret_cast<int32_t*>(base + kOffOrder);
+  int32_t* cost = reinterpret_cast<int32_t*>(base + kOffCost);
+  int32_t* counters = reinterpret_cast<int32_t*>(base + kOffCounters);
+  int32_t* err = reinterpret_cast<int32_t*>(base + kOffError);
+  int64_t* thr = reinterpret_cast<int64_t*>(base + kOffThr);
+  uint8_t* lut = reinterpret_cast<uint8_t*>(base + kOffLut);
+  int32_t* thr32 = reinterpret_cast<int32_t*>(base + kOffThr32);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  noalloc_prepare_kernel<<<1, 256, 0, st>>>(g_noalloc_tables, thr, lut, thr32, counters, err);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess)
+    e = launch_schedule_raw(T, offsets, B, ts, mode, ncand, rows, cost, order, counters, err, st);
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.uvqk = uvqk;
+  a.av = av;
+  a.rows = rows;
+  a.order = order;
+  a.ts = ts;
+  a.thresholds = thr;
+  a.time_lut = lut;
+  a.thr32 = thr32;
+  a.lut_exact = c.time_log_div > 0.2232 ? 1 : 0;
+  a.rab_pos = rab_pos;
+  a.rab_time = rab_time;
+  a.counters = counters;
+  a.error = err;
+  a.T = T;
+  a.d = c.d_model;
+  a.H = c.num_heads;
+  a.hd = c.head_dim;
+  a.pos_clamp = c.pos_clamp;
+  a.time_buckets = c.time_buckets;
+  a.n_norm_fixed = c.n_norm;
+  a.num_pairs = int((T + 2 * kTile - 1) / (2 * kTile));
+  if (e == cudaSuccess) e = launch_attention_tc(a, st, false);
+  if (e == cudaSuccess && device_error != nullptr)
+    e = cudaMemcpyAsync(device_error, err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}

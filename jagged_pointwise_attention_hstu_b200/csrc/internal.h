@@ -111,6 +111,10 @@ namespace hstu {
 cudaError_t launch_schedule(const hstu_handle_s* h, int64_t T, const int32_t* offsets, int32_t B,
                             const int64_t* ts, int mask_mode, const int32_t* ncand,
                             cudaStream_t st);
+// The same schedule into caller-given scratch; counters[0..3] must already be zero.
+cudaError_t launch_schedule_raw(int64_t T, const int32_t* offsets, int32_t B, const int64_t* ts,
+                                int mask_mode, const int32_t* ncand, RowInfo* rows, int32_t* cost,
+                                int32_t* order, int32_t* counters, int32_t* err, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* x, void* xb, int64_t n, cudaStream_t st);
 
 // gemm_tc.cu

@@ -147,6 +147,21 @@ cudaError_t launch_schedule(const hstu_handle_s* h, int64_t T, const int32_t* of
   return cudaGetLastError();
 }
 
+cudaError_t launch_schedule_raw(int64_t T, const int32_t* offsets, int32_t B, const int64_t* ts,
+                                int mask_mode, const int32_t* ncand, RowInfo* rows, int32_t* cost,
+                                int32_t* order, int32_t* counters, int32_t* err, cudaStream_t st) {
+  const int64_t n = (T > int64_t(B) + 1) ? T : int64_t(B) + 1;
+  const int threads = 256;
+  const unsigned blocks = unsigned((n + threads - 1) / threads);
+  rows_kernel<<<blocks, threads, 0, st>>>(offsets, B, T, ncand, mask_mode == HSTU_MASK_MFALCON,
+                                          ts, rows, counters, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || T == 0) return e;
+  const int32_t npairs = int32_t((T + 2 * kTile - 1) / (2 * kTile));
+  order_kernel<<<1, 1024, 0, st>>>(rows, T, npairs, cost, order, counters);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_cast_bf16(const float* x, void* xb, int64_t n, cudaStream_t st) {
   // n is a multiple of 4 (d is a multiple of 16)
   const int64_t n4 = n / 4;

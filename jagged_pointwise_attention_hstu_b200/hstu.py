@@ -91,6 +91,9 @@ def load() -> ctypes.CDLL:
                                                  c_void_p, c_void_p, c_void_p, c_void_p]),
         "hstu_debug_umma_tile": (c_int, [c_int32, c_void_p, c_void_p, c_void_p, c_int32,
                                          c_int32]),
+        "hstu_attention_noalloc": (c_int, [POINTER(hstu_config), c_void_p, c_int64, c_void_p,
+                                           c_int32, c_void_p, c_int, c_void_p, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_void_p]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -203,6 +206,19 @@ def hstu_debug_attention_buckets(handle, total_tokens: int, seq_offsets, num_use
 def hstu_debug_umma_tile(mode: int, a, b, c, n: int, k: int) -> None:
     _check(load().hstu_debug_umma_tile(mode, _ptr(a), _ptr(b), _ptr(c), n, k),
            "hstu_debug_umma_tile")
+
+
+HSTU_NOALLOC_MAX_TOKENS = 65536
+
+
+def hstu_attention_noalloc(cfg: hstu_config, uvqk, total_tokens: int, seq_offsets, num_users: int,
+                           timestamps, mask_mode: int, num_candidates, rab_pos, rab_time, av,
+                           device_error=None, stream=None) -> None:
+    _check(load().hstu_attention_noalloc(ctypes.byref(cfg), _ptr(uvqk), total_tokens,
+                                         _ptr(seq_offsets), num_users, _ptr(timestamps), mask_mode,
+                                         _ptr(num_candidates), _ptr(rab_pos), _ptr(rab_time),
+                                         _ptr(av), _ptr(device_error), _stream_ptr(stream)),
+           "hstu_attention_noalloc")
 
 
 KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2")
