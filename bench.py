@@ -37,6 +37,40 @@ METRIC = "HSTU layer fwd tokens/s (jagged) and attention TFLOP/s as % of B200 BF
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def rank_batch(w, rank, num_layers=None):
+    """The users of one rank: rank r draws its own seeded batch of workload w
+    (weak scaling; ranks share no data, so the data path has no collective)."""
+    return wl.make_batch(w, seed_offset=rank, num_layers=num_layers)
+
+
+def _reduce(x, world, device, op):
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a per-rank number over all ranks (every rank calls it, in the
+    same order); the identity on one rank."""
+    import torch.distributed as dist
+    return _reduce(x, world, device, dist.ReduceOp.MAX)
+
+
+def sum_over_ranks(x, world, device=None):
+    """Sum of a per-rank number over all ranks; the identity on one rank."""
+    import torch.distributed as dist
+    return _reduce(x, world, device, dist.ReduceOp.SUM)
+
+
+def weak_scaling_value(units_all_ranks, ms_max):
+    """Whole-job throughput: the units of every rank over the slowest rank's time."""
+    return units_all_ranks / (ms_max / 1e3)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -46,6 +80,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profiling aid: draw only the first N layers (default: all of the "
+                         "workload's layers; per-layer kernels and their sizes are unchanged)")
     return ap.parse_args()
 
 
@@ -236,7 +273,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     w = wl.WORKLOADS[args.workload]
-    batch = wl.make_batch(w, seed_offset=rank)       # weak scaling: each rank its own users
+    batch = rank_batch(w, rank, num_layers=args.layers)
     L = len(batch.layers)
     T = batch.total_tokens
     cfg = runtime.config_for(w, T, batch.num_users)
@@ -279,13 +316,10 @@ def main():
     hstu.hstu_set_kernel_timing(handle.h, False)
     if handle.device_error():
         raise RuntimeError("device error during the timed region")
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     units_per_rank = T * L
-    value = world * units_per_rank / (ms_max / 1e3)
+    units_all = sum_over_ranks(units_per_rank, world, dev)
+    value = weak_scaling_value(units_all, ms_max)
 
     # ---------------- end to end through the C ABI with host buffers
     e2e = None
@@ -320,12 +354,8 @@ def main():
         e2.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ms_e2e = s2.elapsed_time(e2) / args.steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * units_per_rank / (ms_e2e / 1e3), "unit": "tokens/s",
+        ms_e2e = max_over_ranks(s2.elapsed_time(e2) / args.steps, world, dev)
+        e2e = {"value": weak_scaling_value(units_all, ms_e2e), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ms_e2e}
 

@@ -1,5 +1,5 @@
-// Jagged scheduler: per-token row facts, input validation and the q-tile
-// work order of the attention kernels.
+// Jagged scheduler: per-token row facts, input validation and the work order
+// of the attention kernels (pairs of adjacent query tiles).
 //
 // The batch is jagged (per-user sequences packed without padding; blog
 // "Generative Recommendation 16: HSTU", item 1 "Ragged/Jagged kernel").  Query
@@ -9,9 +9,11 @@
 //   [r0, r0 + 128)             (the diagonal tile)
 // because later users in the tile start inside it and a candidate of the first
 // user sees only that user's history and itself (ltzyclt blog, section 5.2,
-// M-FALCON).  Every other key tile is fully masked and never visited.  The
-// q-tiles are then ordered by descending cost (key tiles visited), a longest-
-// processing-time-first order that keeps the power-law lengths balanced.
+// M-FALCON).  Every other key tile is fully masked and never visited.  A work
+// item is a pair of adjacent query tiles (2p, 2p+1), which visits the union of
+// both tiles' key ranges; the pairs are ordered by descending cost (key tiles
+// visited), a longest-processing-time-first order that keeps the power-law
+// lengths balanced.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
