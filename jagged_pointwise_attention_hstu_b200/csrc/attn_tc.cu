@@ -116,6 +116,9 @@ struct AttnLayout {
   static_assert(kTileBytes % 1024 == 0, "tile stride alignment");
   static_assert(kKts % 128 == 0, "timestamp stage alignment");
   static_assert(kBars % 8 == 0, "mbarrier alignment");
+  // the O tile of query tile 0 (1) is staged for its TMA store in the K (V) ring
+  static constexpr uint32_t kOStageBytes = uint32_t(HD) * 512;   // HD / 32 boxes of 128 x 128 B
+  static_assert(kOStageBytes <= NSK * kTileBytes && kOStageBytes <= NSV * kTileBytes, "O staging");
   static_assert(smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
 };
 
@@ -337,6 +340,7 @@ __device__ __forceinline__ void score_tile(uint32_t taddr, Row& R, const float* 
 template <int HD, bool RECORD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_ts,
+                   const __grid_constant__ CUtensorMap tm_o,
                    const AttnParams p) {
   using L = AttnLayout<HD>;
   constexpr int NSK = L::NSK;
@@ -360,8 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + NSV;
   uint64_t* s_full = v_empty + NSV;  // [2] one per query tile
   uint64_t* p_full = s_full + 2;     // [2]
-  uint64_t* o_full = p_full + 2;
-  uint64_t* t_full = o_full + 1;     // [NST] key timestamps of a tile landed
+  uint64_t* o_full = p_full + 2;     // [2] every product of a query tile is done
+  uint64_t* drained = o_full + 2;    // every MMA of the CTA is done
+  uint64_t* t_full = drained + 1;    // [NST] key timestamps of a tile landed
   uint64_t* t_empty = t_full + NST;  // [NST] every row-group warp is done with them
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + NST);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -395,7 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 128);
     }
-    mbar_init(o_full, 1);
+    mbar_init(&o_full[0], 1);
+    mbar_init(&o_full[1], 1);
+    mbar_init(drained, 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&t_full[s], 1);
       mbar_init(&t_empty[s], 4 * nq);   // the warps of every row group that has rows
@@ -508,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (q == nq - 1) umma_commit(&k_empty[s]);
         return true;
       };
+      bool o_done[2] = {false, false};
       for (int q = 0; ok && q < nq; ++q) ok = issue_qk(q, 0);
       for (int j = 0; ok && j < n_kt; ++j) {
         const int s = j % NSV;
@@ -522,13 +530,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     (j > 0 || kk > 0));
           }
           if (q == nq - 1) umma_commit(&v_empty[s]);
+          if (j + 1 == n_kt) {
+            umma_commit(&o_full[q]);
+            o_done[q] = true;
+          }
           // S_q is rewritten only after P_q V_j (issued just above, executed in order)
           if (j + 1 < n_kt && !issue_qk(q, j + 1)) ok = false;
         }
       }
       if (!ok) *abort_flag = 1;
-      umma_commit(o_full);   // also drains: fires once every MMA above is done
-      mbar_wait(o_full, 0);
+      for (int q = 0; q < nq; ++q)
+        if (!o_done[q]) umma_commit(&o_full[q]);   // release the row groups on an abort
+      umma_commit(drained);   // fires once every MMA above is done
+      mbar_wait(drained, 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ row groups
@@ -679,27 +693,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    bool ok = aborted ? false : mbar_wait(o_full, 0);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && q < nq) {
-      tc_fence_after();
+    // ---- O_q / n_norm -> shared memory (128-byte swizzled boxes of 32 rows x 32
+    // columns, one set per warp) -> TMA store, which clips the rows past T.  Once
+    // o_full[q] fired, no MMA reads the ring that stages this tile any more: the K
+    // ring for query tile 0 (every QK product precedes the last PV of tile 0), the
+    // V ring for query tile 1 (its last PV is the last MMA).
+    if (q < nq) {
+      bool ok = aborted ? false : mbar_wait(&o_full[q], 0);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        uint8_t* stage = smem + (q == 0 ? L::kK : L::kV) + wq * 4096;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO(q) + lane_off + c * 32, r);
-        tmem_ld_wait();
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.av + i * d + h * HD + c * 32);
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO(q) + lane_off + c * 32, r);
+          tmem_ld_wait();
+          const uint32_t row_addr = smem_u32(stage + c * 16384 + lane * 128);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(r[4 * e + 0]) * inv_nn,
-                                 __uint_as_float(r[4 * e + 1]) * inv_nn,
-                                 __uint_as_float(r[4 * e + 2]) * inv_nn,
-                                 __uint_as_float(r[4 * e + 3]) * inv_nn);
+            st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4), __uint_as_float(r[4 * e + 0]) * inv_nn,
+                         __uint_as_float(r[4 * e + 1]) * inv_nn,
+                         __uint_as_float(r[4 * e + 2]) * inv_nn,
+                         __uint_as_float(r[4 * e + 3]) * inv_nn);
         }
+        fence_proxy_async_smem();   // make the stores visible to the TMA unit
+        __syncwarp();
+        if (lane == 0) {
+          for (int c = 0; c < HD / 32; ++c)
+            tma_store_2d(&tm_o, stage + c * 16384, h * HD + c * 32, (qt0 + q) * 128 + wq * 32);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        __syncwarp();
+      } else {
+        *abort_flag = 1;
       }
-    } else if (!ok) {
-      *abort_flag = 1;
     }
   }
 
@@ -715,11 +744,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int HD, bool RECORD>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<HD>;
-  CUtensorMap tm, tm_ts;
+  CUtensorMap tm, tm_ts, tm_o;
   if (!make_tmap_2d_bf16(&tm, a.uvqk, uint64_t(4 * a.d), uint64_t(a.T), uint64_t(4 * a.d) * 2,
                          64, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_1d_i64(&tm_ts, a.ts, uint64_t(a.T), 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_f32_sw128(&tm_o, a.av, uint64_t(a.d), uint64_t(a.T), uint64_t(a.d) * 4, 32, 32))
+    return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, RECORD>,
@@ -752,7 +783,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   p.dump_tidx = a.dump_tidx;
   p.dump_vis = a.dump_vis;
   const int64_t grid = int64_t(a.num_pairs) * a.H;
-  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::smem_bytes(a.pos_clamp), st>>>(tm, tm_ts, p);
+  attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::smem_bytes(a.pos_clamp), st>>>(tm, tm_ts, tm_o, p);
   return cudaGetLastError();
 }
 

@@ -178,6 +178,9 @@ cudaError_t run_umma_tile(int mode, const void* a, const void* b, float* c, int 
 // tensor maps (hstu_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// fp32 [outer, inner] row-major, 128-byte swizzle (box_inner * 4 <= 128).
+bool make_tmap_2d_f32_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_1d_i64(CUtensorMap* m, const void* base, uint64_t n, uint32_t box);
 
 }  // namespace hstu
