@@ -116,9 +116,9 @@ struct AttnLayout {
   static_assert(kTileBytes % 1024 == 0, "tile stride alignment");
   static_assert(kKts % 128 == 0, "timestamp stage alignment");
   static_assert(kBars % 8 == 0, "mbarrier alignment");
-  // the O tile of query tile 0 (1) is staged for its TMA store in the K (V) ring
-  static constexpr uint32_t kOStageBytes = uint32_t(HD) * 512;   // HD / 32 boxes of 128 x 128 B
-  static_assert(kOStageBytes <= NSK * kTileBytes && kOStageBytes <= NSV * kTileBytes, "O staging");
+  // O of query tile q is staged for its TMA stores in Q_q's tile, in two rounds:
+  // per warp a quarter of the tile holds HD / 64 boxes of 32 rows x 32 fp32 columns
+  static_assert((kTileBytes / 4) % 4096 == 0 && (kTileBytes / 4) / 4096 == HD / 64, "O staging");
   static_assert(smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
 };
 
@@ -365,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + NSV;  // [2] one per query tile
   uint64_t* p_full = s_full + 2;     // [2]
   uint64_t* o_full = p_full + 2;     // [2] every product of a query tile is done
-  uint64_t* drained = o_full + 2;    // every MMA of the CTA is done
-  uint64_t* t_full = drained + 1;    // [NST] key timestamps of a tile landed
+  uint64_t* drained = o_full + 2;    // [2] every MMA of one issuer is done
+  uint64_t* t_full = drained + 2;    // [NST] key timestamps of a tile landed
   uint64_t* t_empty = t_full + NST;  // [NST] every row-group warp is done with them
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + NST);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -390,11 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < NSK; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_empty[s], nq);   // one commit per MMA issuer
     }
     for (int s = 0; s < NSV; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&v_empty[s], nq);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -402,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&o_full[0], 1);
     mbar_init(&o_full[1], 1);
-    mbar_init(drained, 1);
+    mbar_init(&drained[0], 1);
+    mbar_init(&drained[1], 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&t_full[s], 1);
       mbar_init(&t_empty[s], 4 * nq);   // the warps of every row group that has rows
@@ -423,18 +424,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tO = [&](int q) -> uint32_t { return tmem_base + 256 + q * HD; };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ Q and K loads
+    // ------------------------------------------------------------ Q, K and key timestamp loads
     if (lane == 0) {
       prefetch_tmap(&tm);
+      prefetch_tmap(&tm_ts);
       mbar_arrive_expect_tx(q_full, nq * L::kTileBytes);
       for (int q = 0; q < nq; ++q)
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
           tma_load_2d(smem + L::kQ + q * L::kTileBytes + b * 16384, &tm, q_full,
                       2 * d + h * HD + b * 64, (qt0 + q) * 128);
-      bool issued[NSK];
-      uint32_t issued_ph[NSK];
+      bool issued[NSK], t_issued[NST];
+      uint32_t issued_ph[NSK], t_issued_ph[NST];
       for (int s = 0; s < NSK; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int s = 0; s < NST; ++s) t_issued[s] = false, t_issued_ph[s] = 0;
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int s = j % NSK;
         const uint32_t ph = (j / NSK) & 1;
@@ -446,13 +449,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                       3 * d + h * HD + b * 64, key_tile(j) * 128);
         issued[s] = true;
         issued_ph[s] = ph;
+        // the tile's key timestamps (a deeper ring: the row groups classify ahead)
+        const int st = j % NST;
+        const uint32_t tph = (j / NST) & 1;
+        if (!mbar_wait(&t_empty[st], tph ^ 1)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(&t_full[st], 128 * 8);
+        tma_load_1d(s_kts + st * 128, &tm_ts, &t_full[st], key_tile(j) * 128);
+        t_issued[st] = true;
+        t_issued_ph[st] = tph;
       }
       mbar_wait(q_full, 0);
       for (int s = 0; s < NSK; ++s)
         if (issued[s]) mbar_wait(&k_full[s], issued_ph[s]);
+      for (int s = 0; s < NST; ++s)
+        if (t_issued[s]) mbar_wait(&t_full[s], t_issued_ph[s]);
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ V + key timestamp loads
+    // ------------------------------------------------------------ V loads
     if (lane == 0) {
       bool issued[NSV];
       uint32_t issued_ph[NSV];
@@ -472,38 +485,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < NSV; ++s)
         if (issued[s]) mbar_wait(&v_full[s], issued_ph[s]);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ key timestamp loads
-    if (lane == 0) {
-      prefetch_tmap(&tm_ts);
-      bool issued[NST];
-      uint32_t issued_ph[NST];
-      for (int s = 0; s < NST; ++s) issued[s] = false, issued_ph[s] = 0;
-      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
-        const int s = j % NST;
-        const uint32_t ph = (j / NST) & 1;
-        if (!mbar_wait(&t_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&t_full[s], 128 * 8);
-        tma_load_1d(s_kts + s * 128, &tm_ts, &t_full[s], key_tile(j) * 128);
-        issued[s] = true;
-        issued_ph[s] = ph;
-      }
-      for (int s = 0; s < NST; ++s)
-        if (issued[s]) mbar_wait(&t_full[s], issued_ph[s]);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issue, one thread per
+    // query tile (warp 1: tile 0, warp 3: tile 1).  Two issuers keep the tensor pipe fed while
+    // either one waits for its row group: an issuing thread that stops for a wait lets the
+    // pipe drain.
+    const int q = warp == 1 ? 0 : 1;
+    if (lane == 0 && q < nq) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, HD, false, true);
       bool ok = mbar_wait(q_full, 0);
       tc_fence_after();
-      // S_q = Q_q K_j^T; after the last query tile of key tile j the K stage is released
-      auto issue_qk = [&](int q, int j) -> bool {
+      const uint32_t sQ = smem_u32(smem + L::kQ + q * L::kTileBytes);
+      // S_q = Q_q K_j^T; the K stage is released once every issuer's product has read it
+      auto issue_qk = [&](int j) -> bool {
         const int s = j % NSK;
         if (!mbar_wait(&k_full[s], (j / NSK) & 1)) return false;
         tc_fence_after();
-        const uint32_t sQ = smem_u32(smem + L::kQ + q * L::kTileBytes);
         const uint32_t sK = smem_u32(smem + L::kK + s * L::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
@@ -512,37 +510,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                   idesc_qk, kk > 0);
         }
         umma_commit(&s_full[q]);
-        if (q == nq - 1) umma_commit(&k_empty[s]);
+        umma_commit(&k_empty[s]);
         return true;
       };
-      bool o_done[2] = {false, false};
-      for (int q = 0; ok && q < nq; ++q) ok = issue_qk(q, 0);
+      if (ok) ok = issue_qk(0);
+      bool o_done = false;
       for (int j = 0; ok && j < n_kt; ++j) {
         const int s = j % NSV;
         if (!mbar_wait(&v_full[s], (j / NSV) & 1)) { ok = false; break; }
+        if (!mbar_wait(&p_full[q], j & 1)) { ok = false; break; }
+        tc_fence_after();
         const uint32_t sV = smem_u32(smem + L::kV + s * L::kTileBytes);
-        for (int q = 0; ok && q < nq; ++q) {
-          if (!mbar_wait(&p_full[q], j & 1)) { ok = false; break; }
-          tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            umma_ts(tO(q), tS(q) + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
-                    (j > 0 || kk > 0));
-          }
-          if (q == nq - 1) umma_commit(&v_empty[s]);
-          if (j + 1 == n_kt) {
-            umma_commit(&o_full[q]);
-            o_done[q] = true;
-          }
-          // S_q is rewritten only after P_q V_j (issued just above, executed in order)
-          if (j + 1 < n_kt && !issue_qk(q, j + 1)) ok = false;
+        for (int kk = 0; kk < 8; ++kk) {
+          umma_ts(tO(q), tS(q) + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
+                  (j > 0 || kk > 0));
         }
+        umma_commit(&v_empty[s]);
+        if (j + 1 == n_kt) {
+          umma_commit(&o_full[q]);
+          o_done = true;
+        }
+        // S_q is rewritten only after P_q V_j (issued just above, executed in order)
+        if (j + 1 < n_kt && !issue_qk(j + 1)) ok = false;
       }
       if (!ok) *abort_flag = 1;
-      for (int q = 0; q < nq; ++q)
-        if (!o_done[q]) umma_commit(&o_full[q]);   // release the row groups on an abort
-      umma_commit(drained);   // fires once every MMA above is done
-      mbar_wait(drained, 0);
+      if (!o_done) umma_commit(&o_full[q]);   // release the row group on an abort
+      umma_commit(&drained[q]);              // fires once every MMA of this issuer is done
+      mbar_wait(&drained[q], 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ row groups
@@ -694,38 +689,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- O_q / n_norm -> shared memory (128-byte swizzled boxes of 32 rows x 32
-    // columns, one set per warp) -> TMA store, which clips the rows past T.  Once
-    // o_full[q] fired, no MMA reads the ring that stages this tile any more: the K
-    // ring for query tile 0 (every QK product precedes the last PV of tile 0), the
-    // V ring for query tile 1 (its last PV is the last MMA).
+    // columns, per warp) -> TMA stores, which clip the rows past T.  Once o_full[q]
+    // fired, every MMA of this query tile is done, so Q_q's tile is free to stage in.
     if (q < nq) {
       bool ok = aborted ? false : mbar_wait(&o_full[q], 0);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        uint8_t* stage = smem + (q == 0 ? L::kK : L::kV) + wq * 4096;
+        uint8_t* stage = smem + L::kQ + q * L::kTileBytes + wq * (L::kTileBytes / 4);
+        constexpr int kBoxes = HD / 64;   // boxes per round; two rounds cover HD columns
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO(q) + lane_off + c * 32, r);
-          tmem_ld_wait();
-          const uint32_t row_addr = smem_u32(stage + c * 16384 + lane * 128);
+        for (int rd = 0; rd < 2; ++rd) {
+#pragma unroll 1
+          for (int cb = 0; cb < kBoxes; ++cb) {
+            uint32_t r[32];
+            tmem_ld32(tO(q) + lane_off + (rd * kBoxes + cb) * 32, r);
+            tmem_ld_wait();
+            const uint32_t row_addr = smem_u32(stage + cb * 4096 + lane * 128);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4), __uint_as_float(r[4 * e + 0]) * inv_nn,
-                         __uint_as_float(r[4 * e + 1]) * inv_nn,
-                         __uint_as_float(r[4 * e + 2]) * inv_nn,
-                         __uint_as_float(r[4 * e + 3]) * inv_nn);
+            for (int e = 0; e < 8; ++e)
+              st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4),
+                           __uint_as_float(r[4 * e + 0]) * inv_nn,
+                           __uint_as_float(r[4 * e + 1]) * inv_nn,
+                           __uint_as_float(r[4 * e + 2]) * inv_nn,
+                           __uint_as_float(r[4 * e + 3]) * inv_nn);
+          }
+          fence_proxy_async_smem();   // make the stores visible to the TMA unit
+          __syncwarp();
+          if (lane == 0) {
+            for (int cb = 0; cb < kBoxes; ++cb)
+              tma_store_2d(&tm_o, stage + cb * 4096, h * HD + (rd * kBoxes + cb) * 32,
+                           (qt0 + q) * 128 + wq * 32);
+            bulk_commit_group();
+            bulk_wait_group_read0();   // the boxes are reused by the next round
+          }
+          __syncwarp();
         }
-        fence_proxy_async_smem();   // make the stores visible to the TMA unit
-        __syncwarp();
-        if (lane == 0) {
-          for (int c = 0; c < HD / 32; ++c)
-            tma_store_2d(&tm_o, stage + c * 16384, h * HD + c * 32, (qt0 + q) * 128 + wq * 32);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        __syncwarp();
       } else {
         *abort_flag = 1;
       }
