@@ -67,6 +67,10 @@ using namespace sm100;
 constexpr int kMaxPosEntries = 4097;   // pos_clamp <= 4096
 constexpr int kMaxTimeBuckets = 256;
 constexpr int kThreads = 384;
+// The shared copy of rab_pos is padded on both sides with its end values, so
+// that any relative position pos_rel - column in [-kPosPad, clamp + kPosPad]
+// reads the clamped entry without a min/max.
+constexpr int kPosPad = 130;
 constexpr int kFast = 0, kMed = 1, kCut = 2, kAny = 3, kGen = 4, kZero = 5;
 
 struct AttnParams {
@@ -107,9 +111,10 @@ struct AttnLayout {
   static constexpr uint32_t kAnyTab = kLut + 128;                    // int4 [128]
   static constexpr uint32_t kRabTime = kAnyTab + 128 * 16;
   static constexpr uint32_t kBars = kRabTime + kMaxTimeBuckets * 4;
-  static constexpr uint32_t kRabPos = kBars + 256;                   // float [clamp + 1]
+  // float [clamp + 1 + 2 kPosPad]: rab_pos[clamp(k, 0, clamp)] at k + kPosPad
+  static constexpr uint32_t kRabPos = kBars + 256;
   static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
-    return kRabPos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16 + 1024;
+    return kRabPos + ((uint32_t(clamp + 1 + 2 * kPosPad) * 4 + 15) / 16) * 16 + 1024;
   }
   // every TMA destination starts on a 1024-byte (swizzled tiles) or 128-byte boundary
   static_assert(kQ % 1024 == 0 && kK % 1024 == 0 && kV % 1024 == 0, "tile alignment");
@@ -157,7 +162,7 @@ struct Row {
   int64_t ti, cut, cut_last;
   float hc, hc_hi, hc_lo;               // half-bias constants of the fast paths
   float hc2, hc3;                       // kCut: half-bias of buckets b - 2, b - 3
-  int th1, th2, th3;                    // kMed/kCut: a gap below th_m drops a bucket
+  int j1, j2, j3;                       // kMed/kCut: keys from column j_m on drop one more bucket
   uint32_t ti_lo;                       // low 32 bits of t_i (kMed, kCut, kAny)
 };
 
@@ -179,23 +184,20 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
     float add = R.hc;
     int tb = R.b;
     if constexpr (MODE != kFast) {
-      const int dd = int(R.ti_lo - uint32_t(tk));   // the gap; in [0, 2^31) on these paths
-      const bool d1 = dd < R.th1;
+      // timestamps are sorted inside the user: the gap shrinks as the column grows
+      const bool d1 = jr >= R.j1;
       add = d1 ? R.hc_lo : R.hc;
       if constexpr (RECORD) tb = R.b - (d1 ? 1 : 0);
       if constexpr (MODE == kCut) {
-        const bool d2 = dd < R.th2;
-        const bool d3 = dd < R.th3;
+        const bool d2 = jr >= R.j2;
+        const bool d3 = jr >= R.j3;
         add = d2 ? (d3 ? R.hc3 : R.hc2) : add;
         if constexpr (RECORD) tb -= (d2 ? 1 : 0) + (d3 ? 1 : 0);
       }
     }
-    int pidx = clamp;
-    if constexpr (!PC) {
-      pidx = min(R.pos_rel - jr, clamp);
-      add = fmaf(0.5f, s_rp[pidx], add);
-    }
+    if constexpr (!PC) add = fmaf(0.5f, s_rp[-jr], add);
     if constexpr (RECORD) {
+      const int pidx = PC ? clamp : min(R.pos_rel - jr, clamp);
       if (rec.on) {
         const int64_t at = rec.i * rec.T + rec.kb + jr;
         rec.pidx[at] = pidx;
@@ -215,8 +217,8 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
     const int4 ent = reinterpret_cast<const int4*>(s_lut)[idx];   // {thr, rt_lo, rt_hi, cand}
     const bool up = int(dd) >= ent.x;
     const float rt = __int_as_float(up ? ent.z : ent.y);
-    const int pidx = min(max(R.pos_rel - jr, 0), clamp);
     if constexpr (RECORD) {
+      const int pidx = min(max(R.pos_rel - jr, 0), clamp);
       if (rec.on && rec.kb + jr < rec.T) {
         const int64_t at = rec.i * rec.T + rec.kb + jr;
         rec.pidx[at] = pidx;
@@ -224,14 +226,14 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
         rec.vis[at] = vis ? 1 : 0;
       }
     }
-    const float hh = 0.5f * (acc + s_rp[pidx] + rt);
+    const float hh = 0.5f * (acc + s_rp[-jr] + rt);
     return vis ? silu_half(hh) : 0.0f;
   } else {
     if (jr >= R.lo_rel && jr <= R.i_rel) walk_to(R.b, R.cut, tk, R.ti, s_thr);
-    const int dp = R.pos_rel - jr;
-    const int pidx = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
     const bool vis = (unsigned(jr - R.lo_rel) < unsigned(R.hi_rel - R.lo_rel)) || jr == R.i_rel;
     if constexpr (RECORD) {
+      const int dp = R.pos_rel - jr;
+      const int pidx = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
       if (rec.on && rec.kb + jr < rec.T) {
         const int64_t at = rec.i * rec.T + rec.kb + jr;
         rec.pidx[at] = pidx;
@@ -239,7 +241,7 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
         rec.vis[at] = vis ? 1 : 0;
       }
     }
-    const float sc = acc + s_rp[pidx] + s_rt[R.b];
+    const float sc = acc + s_rp[-jr] + s_rt[R.b];
     return vis ? silu_half(0.5f * sc) : 0.0f;
   }
 }
@@ -255,7 +257,7 @@ __device__ __forceinline__ void score_chunk(const uint32_t (&r)[16], int c, uint
 #pragma unroll
   for (int e = 0; e < 16; e += 2) {
     int64_t t0 = 0, t1 = 0;
-    if constexpr (MODE != kFast) {
+    if constexpr (MODE == kAny || MODE == kGen) {
       const longlong2 kk = k2[e >> 1];
       t0 = kk.x;
       t1 = kk.y;
@@ -547,7 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
-    for (int k = threadIdx.x - 128; k <= clamp; k += 256) s_rab_pos[k] = p.rab_pos[k];
+    for (int k = threadIdx.x - 128; k <= clamp + 2 * kPosPad; k += 256)
+      s_rab_pos[k] = p.rab_pos[min(max(k - kPosPad, 0), clamp)];
     for (int k = threadIdx.x - 128; k < nb; k += 256) {
       s_rab_time[k] = p.rab_time[k];
       s_thr[k] = p.thresholds[k];
@@ -623,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mode;
       if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
       else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
-      else if (__all_sync(0xffffffffu, full && lev <= 1 && narrow)) mode = kMed;
-      else if (__all_sync(0xffffffffu, full && lev <= 3 && narrow)) mode = kCut;
+      else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
+      else if (__all_sync(0xffffffffu, full && lev <= 3)) mode = kCut;
       else if (p.lut_exact &&
                __all_sync(0xffffffffu, (full || (history && lo <= kb)) && narrow))
         mode = kAny;
@@ -633,15 +636,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mode == kFast || mode == kMed || mode == kCut) {
         // R.b = bucket of the tile's first key (the largest gap); a gap below
         // thr[R.b - m + 1] drops the bucket below R.b - m + 1
-        const float rp_c = pc ? s_rab_pos[clamp] : 0.0f;
+        const float rp_c = pc ? s_rab_pos[kPosPad + clamp] : 0.0f;
         const int b0 = R.b;
         R.hc = 0.5f * (rp_c + s_rab_time[b0]);
         R.hc_lo = 0.5f * (rp_c + s_rab_time[max(b0 - 1, 0)]);
         R.hc2 = 0.5f * (rp_c + s_rab_time[max(b0 - 2, 0)]);
         R.hc3 = 0.5f * (rp_c + s_rab_time[max(b0 - 3, 0)]);
-        R.th1 = s_thr32[b0];
-        R.th2 = s_thr32[max(b0 - 1, 0)];
-        R.th3 = s_thr32[max(b0 - 2, 0)];
+        if (mode != kFast) {
+          // first column whose gap is below thr[b0 - m + 1]: the count of keys with
+          // t_j <= t_i - thr[b0 - m + 1] (the tile's timestamps are sorted)
+          const int64_t c1 = R.ti - s_thr[b0];
+          const int64_t c2 = R.ti - s_thr[max(b0 - 1, 0)];
+          const int64_t c3 = R.ti - s_thr[max(b0 - 2, 0)];
+          int p1 = 0, p2 = 0, p3 = 0;
+#pragma unroll
+          for (int step = 64; step > 0; step >>= 1) {
+            if (kts[p1 + step - 1] <= c1) p1 += step;
+            if (mode == kCut) {
+              if (kts[p2 + step - 1] <= c2) p2 += step;
+              if (kts[p3 + step - 1] <= c3) p3 += step;
+            }
+          }
+          // seven halvings leave p in [0, 127]; one more compare completes the count
+          R.j1 = p1 + (kts[p1] <= c1 ? 1 : 0);
+          R.j2 = p2 + (kts[p2] <= c2 ? 1 : 0);
+          R.j3 = p3 + (kts[p3] <= c3 ? 1 : 0);
+        }
       }
       Record rec;
       rec.pidx = p.dump_pidx;
@@ -661,21 +681,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tS(q) + lane_off;
+      // rp_row[-column] = rab_pos[clamp(pos_rel - column, 0, clamp)]
+      const float* rp_row = s_rab_pos + kPosPad + R.pos_rel;
       if (mode == kZero) {
         zero_tile<RECORD>(taddr, rec);
       } else if (mode == kFast) {
-        if (pc) score_tile<kFast, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
-        else score_tile<kFast, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        if (pc) score_tile<kFast, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kFast, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else if (mode == kMed) {
-        if (pc) score_tile<kMed, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
-        else score_tile<kMed, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        if (pc) score_tile<kMed, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kMed, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else if (mode == kCut) {
-        if (pc) score_tile<kCut, true, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
-        else score_tile<kCut, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        if (pc) score_tile<kCut, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        else score_tile<kCut, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else if (mode == kAny) {
-        score_tile<kAny, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        score_tile<kAny, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       } else {
-        score_tile<kGen, false, RECORD>(taddr, R, s_rab_pos, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
+        score_tile<kGen, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec);
       }
       tmem_st_wait();
       tc_fence_before();
