@@ -13,7 +13,10 @@
 // 4-stage ring, warp 1 issues 128 x BN x 16 MMAs into one of two tensor-memory
 // accumulators, warps 2-9 drain the other accumulator through the fused
 // epilogue (two warps per tensor-memory lane quarter, each taking half of the
-// columns), so the epilogue of tile t overlaps the MMAs of tile t+1.
+// columns), so the epilogue of tile t overlaps the MMAs of tile t+1.  Each
+// epilogue warp stages 32 rows x 128 bytes of output at a time in its own
+// 128-byte-swizzled shared box and writes it with a TMA store, which clips the
+// rows past M.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -45,7 +48,8 @@ struct GemmLayout {
   static constexpr uint32_t kABytes = 128 * kBK * 2;
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kBarOffset = kStages * kStageBytes;
+  static constexpr uint32_t kOutOffset = kStages * kStageBytes;   // 8 boxes of 4 KB
+  static constexpr uint32_t kBarOffset = kOutOffset + 8 * 4096;
   static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
   static_assert(kABytes % 1024 == 0 && kStageBytes % 1024 == 0, "TMA destinations 1024-aligned");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -61,7 +65,8 @@ constexpr int kGemmThreads = 320;
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
-                   const __grid_constant__ CUtensorMap tma_b, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tma_b,
+                   const __grid_constant__ CUtensorMap tma_out, const GemmParams p) {
   using L = GemmLayout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -169,6 +174,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const int c_begin = ((warp - 2) >> 2) * (BN / 2);
+    uint8_t* box = smem + L::kOutOffset + (warp - 2) * 4096;
+    const uint32_t row_addr = smem_u32(box + lane * 128);
+    // 16-byte chunk e of this thread's 128-byte box row (128-byte swizzle)
+    auto chunk = [&](int e) -> uint32_t { return row_addr + ((e ^ (lane & 7)) << 4); };
+    const bool out_bf16 = p.epi == int(Epi::kSiluSplit) || !p.io_fp32;
+    const int step = out_bf16 ? 64 : 32;   // columns per 128-byte box row
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
@@ -177,55 +188,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int64_t mt = t / n_tiles;
       const int nt = int(t % n_tiles);
       const int64_t grow = mt * 128 + row;
-      const bool valid = grow < p.M;
+      const bool valid = grow < p.M;   // rows past M are computed on zeros and clipped by the store
 #pragma unroll 1
-      for (int c = c_begin; c < c_begin + BN / 2; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + acc * BN + c + (uint32_t(q * 32) << 16), r);
-        tmem_ld_wait();
-        if (!valid) continue;
+      for (int c = c_begin; c < c_begin + BN / 2; c += step) {
         const int col0 = nt * BN + c;
-        const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
-        float v[32];
+        float v[64];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 bb = __ldg(b4 + e);
-          v[4 * e + 0] = __uint_as_float(r[4 * e + 0]) + bb.x;
-          v[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y;
-          v[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z;
-          v[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w;
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !out_bf16) break;
+          uint32_t r[32];
+          tmem_ld32(tmem_base + acc * BN + c + 32 * h + (uint32_t(q * 32) << 16), r);
+          tmem_ld_wait();
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0 + 32 * h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 bb = __ldg(b4 + e);
+            v[32 * h + 4 * e + 0] = __uint_as_float(r[4 * e + 0]) + bb.x;
+            v[32 * h + 4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y;
+            v[32 * h + 4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z;
+            v[32 * h + 4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w;
+          }
         }
         if (p.epi == int(Epi::kSiluSplit)) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
-                                                grow * int64_t(p.N) + col0);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint4 o;
-            o.x = pack_bf16x2(silu_f(v[8 * e + 0]), silu_f(v[8 * e + 1]));
-            o.y = pack_bf16x2(silu_f(v[8 * e + 2]), silu_f(v[8 * e + 3]));
-            o.z = pack_bf16x2(silu_f(v[8 * e + 4]), silu_f(v[8 * e + 5]));
-            o.w = pack_bf16x2(silu_f(v[8 * e + 6]), silu_f(v[8 * e + 7]));
-            dst[e] = o;
-          }
+          for (int e = 0; e < 8; ++e)
+            st_shared_v4_u32(chunk(e), pack_bf16x2(silu_f(v[8 * e + 0]), silu_f(v[8 * e + 1])),
+                             pack_bf16x2(silu_f(v[8 * e + 2]), silu_f(v[8 * e + 3])),
+                             pack_bf16x2(silu_f(v[8 * e + 4]), silu_f(v[8 * e + 5])),
+                             pack_bf16x2(silu_f(v[8 * e + 6]), silu_f(v[8 * e + 7])));
         } else if (p.io_fp32) {
           const float4* res = reinterpret_cast<const float4*>(
               static_cast<const float*>(p.residual) + grow * int64_t(p.N) + col0);
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) +
-                                                  grow * int64_t(p.N) + col0);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float4 x = res[e];
-            dst[e] = make_float4(v[4 * e + 0] + x.x, v[4 * e + 1] + x.y, v[4 * e + 2] + x.z,
-                                 v[4 * e + 3] + x.w);
+            const float4 x = valid ? res[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            st_shared_v4(chunk(e), v[4 * e + 0] + x.x, v[4 * e + 1] + x.y, v[4 * e + 2] + x.z,
+                         v[4 * e + 3] + x.w);
           }
         } else {
           const uint4* res = reinterpret_cast<const uint4*>(
               static_cast<const uint16_t*>(p.residual) + grow * int64_t(p.N) + col0);
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
-                                                grow * int64_t(p.N) + col0);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint4 x = res[e];
+          for (int e = 0; e < 8; ++e) {
+            const uint4 x = valid ? res[e] : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
             uint32_t os[4];
 #pragma unroll
@@ -234,9 +239,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float hi = __uint_as_float(xs[w] & 0xFFFF0000u);
               os[w] = pack_bf16x2(v[8 * e + 2 * w] + lo, v[8 * e + 2 * w + 1] + hi);
             }
-            dst[e] = make_uint4(os[0], os[1], os[2], os[3]);
+            st_shared_v4_u32(chunk(e), os[0], os[1], os[2], os[3]);
           }
         }
+        fence_proxy_async_smem();   // make the stores visible to the TMA unit
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tma_out, box, col0, int32_t(mt * 128 + q * 32));
+          bulk_commit_group();
+          bulk_wait_group_read0();   // the box is refilled by the next step
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
@@ -255,11 +268,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
   using L = GemmLayout<BN>;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, to;
   if (!make_tmap_2d_bf16(&ta, a.a, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K) * 2, kBK, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK, BN))
     return cudaErrorInvalidValue;
+  // output boxes: 32 rows x 128 bytes (64 bf16 or 32 fp32 columns)
+  const bool out_f32 = a.epi == Epi::kBiasResidual && a.io_fp32;
+  const bool ok_o = out_f32 ? make_tmap_2d_f32_sw128(&to, a.out, uint64_t(a.N), uint64_t(a.M),
+                                                     uint64_t(a.N) * 4, 32, 32)
+                            : make_tmap_2d_bf16(&to, a.out, uint64_t(a.N), uint64_t(a.M),
+                                                uint64_t(a.N) * 2, 64, 32);
+  if (!ok_o) return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>,
@@ -280,7 +300,7 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   p.error = error;
   const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
   const int grid = int(tiles < num_sms ? tiles : num_sms);
-  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, p);
+  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, p);
   return cudaGetLastError();
 }
 
