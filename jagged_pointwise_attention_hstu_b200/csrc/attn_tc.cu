@@ -146,10 +146,6 @@ __device__ __forceinline__ void walk_to(int& b, int64_t& cut, int64_t tk, int64_
   }
 }
 
-__device__ __forceinline__ int clamp_i32(int64_t v, int lo, int hi) {
-  return v < lo ? lo : (v > hi ? hi : int(v));
-}
-
 __device__ __forceinline__ float silu_half(float hh) {
   // SiLU(s) with hh = s / 2:  s * sigmoid(s) = hh * (1 + tanh(hh))
   return fmaf(hh, tanh_approx(hh), hh);
@@ -570,14 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(1, 256);
     const uint8_t* s_anyb = reinterpret_cast<const uint8_t*>(s_any);
 
-    const int64_t i = int64_t(qt0 + q) * 128 + row;
+    // token indices fit in int32 (T < 2^31)
+    const int i = (qt0 + q) * 128 + row;
     const bool valid = q < nq && i < p.T;
-    int64_t lo = 0, hi = 0, pos = 0;   // rows past T see nothing
+    int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
     Row R;
     R.ti = 0;
     if (valid) {
       const RowInfo ri = p.rows[i];
-      lo = (ri.lo < 0 || ri.lo > i) ? i : int64_t(ri.lo);
+      lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
       hi = ri.hi;
       pos = ri.pos;
       R.ti = p.ts[i];
@@ -595,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool aborted = false;
 
     for (int j = 0; q < nq && j < n_kt; ++j) {
-      const int64_t kb = int64_t(key_tile(j)) * 128;
+      const int kb = key_tile(j) * 128;
       const int st = j % NST;
       const int64_t* kts = s_kts + st * 128;
       // The key timestamps of tile j come through their own ring, loaded well
@@ -608,12 +605,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       // ---- classify this row for the tile
-      R.lo_rel = clamp_i32(lo - kb, -1, 129);
-      R.hi_rel = clamp_i32(hi - kb, -1, 129);
-      R.i_rel = valid ? clamp_i32(i - kb, -1, 129) : -1;
-      R.pos_rel = clamp_i32(pos - kb, -1, clamp + 129);
-      const bool full = valid && lo <= kb && hi >= kb + 128;
-      const bool posc = (pos - (kb + 127)) >= clamp;
+      R.lo_rel = min(max(lo - kb, -1), 129);
+      R.hi_rel = min(max(hi - kb, -1), 129);
+      R.i_rel = valid ? min(max(i - kb, -1), 129) : -1;
+      R.pos_rel = min(max(pos - kb, -1), clamp + 129);
+      const bool full = valid && lo <= kb && hi - kb >= 128;
+      const bool posc = pos - kb - 127 >= clamp;
       int lev = 99;
       if (full) {
         walk_to(R.b, R.cut, kts[0], R.ti, s_thr);
