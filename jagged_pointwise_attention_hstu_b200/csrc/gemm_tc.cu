@@ -40,6 +40,7 @@ struct GemmParams {
   void* out;
   const void* residual;
   int io_fp32;
+  int out_bf16;         // fp32 out: also store bf16(out) through tma_out2
   int32_t* error;
 };
 
@@ -66,7 +67,8 @@ template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
                    const __grid_constant__ CUtensorMap tma_b,
-                   const __grid_constant__ CUtensorMap tma_out, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap tma_out,
+                   const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
   using L = GemmLayout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -222,8 +224,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const float4 x = valid ? res[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-            st_shared_v4(chunk(e), v[4 * e + 0] + x.x, v[4 * e + 1] + x.y, v[4 * e + 2] + x.z,
-                         v[4 * e + 3] + x.w);
+            v[4 * e + 0] += x.x;
+            v[4 * e + 1] += x.y;
+            v[4 * e + 2] += x.z;
+            v[4 * e + 3] += x.w;
+            st_shared_v4(chunk(e), v[4 * e + 0], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
           }
         } else {
           const uint4* res = reinterpret_cast<const uint4*>(
@@ -250,6 +255,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_wait_group_read0();   // the box is refilled by the next step
         }
         __syncwarp();
+        if (!out_bf16 && p.out_bf16) {
+          // bf16 copy of the 32 fp32 columns: 64-byte box rows, 64-byte swizzle
+          // (16-byte chunk e of row r sits at chunk e ^ ((r / 2) mod 4))
+          const uint32_t row64 = smem_u32(box + lane * 64);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            st_shared_v4_u32(row64 + ((e ^ ((lane >> 1) & 3)) << 4),
+                             pack_bf16x2(v[8 * e + 0], v[8 * e + 1]),
+                             pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                             pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                             pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_out2, box, col0, int32_t(mt * 128 + q * 32));
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          __syncwarp();
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
@@ -268,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 template <int BN>
 cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
   using L = GemmLayout<BN>;
-  CUtensorMap ta, tb, to;
+  CUtensorMap ta, tb, to, to2;
   if (!make_tmap_2d_bf16(&ta, a.a, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K) * 2, kBK, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK, BN))
@@ -280,6 +305,11 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
                             : make_tmap_2d_bf16(&to, a.out, uint64_t(a.N), uint64_t(a.M),
                                                 uint64_t(a.N) * 2, 64, 32);
   if (!ok_o) return cudaErrorInvalidValue;
+  const bool copy = out_f32 && a.out_bf16 != nullptr;
+  to2 = to;   // unused unless copy
+  if (copy && !make_tmap_2d_bf16_sw64(&to2, a.out_bf16, uint64_t(a.N), uint64_t(a.M),
+                                      uint64_t(a.N) * 2, 32, 32))
+    return cudaErrorInvalidValue;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>,
@@ -297,10 +327,11 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   p.out = a.out;
   p.residual = a.residual;
   p.io_fp32 = a.io_fp32;
+  p.out_bf16 = copy ? 1 : 0;
   p.error = error;
   const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
   const int grid = int(tiles < num_sms ? tiles : num_sms);
-  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, p);
+  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, to2, p);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,19 @@ bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_bf16_sw64(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr || outer == 0 || inner == 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_2d_f32_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
   auto fn = encode_fn();
@@ -284,8 +297,11 @@ hstu_status check_weights(const hstu_layer_weights* w) {
 }
 
 // One layer after the schedule is built: f1 -> attention -> LN (.) U -> f2.
+// xb_ready: ws.xb already holds bf16(x) (written by the previous layer's f2);
+// make_xb: f2 also writes bf16(out) to ws.xb for the next layer (fp32 io only).
 hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* ts,
-                      const hstu_layer_weights* w, void* out, cudaStream_t st) {
+                      const hstu_layer_weights* w, void* out, cudaStream_t st, bool xb_ready,
+                      bool make_xb) {
   const hstu_config& c = h->cfg;
   Workspace& ws = h->ws;
   const int d = c.d_model;
@@ -340,8 +356,10 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   }
   const void* xa = x;
   if (io32) {
-    Timed tm(h, kCast, st);
-    e = hstu::launch_cast_bf16(static_cast<const float*>(x), ws.xb, T * d, st);
+    if (!xb_ready) {
+      Timed tm(h, kCast, st);
+      e = hstu::launch_cast_bf16(static_cast<const float*>(x), ws.xb, T * d, st);
+    }
     xa = ws.xb;
   }
   hstu::GemmArgs g1;
@@ -355,6 +373,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   g1.out = ws.uvqk;
   g1.residual = nullptr;
   g1.io_fp32 = 0;
+  g1.out_bf16 = nullptr;
   if (e == cudaSuccess) {
     Timed tm(h, kF1, st);
     e = hstu::launch_gemm_tc(g1, h->num_sms, st, ws.error);
@@ -378,6 +397,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   g2.out = out;
   g2.residual = x;
   g2.io_fp32 = io32 ? 1 : 0;
+  g2.out_bf16 = (io32 && make_xb) ? ws.xb : nullptr;
   if (e == cudaSuccess) {
     Timed tm(h, kF2, st);
     e = hstu::launch_gemm_tc(g2, h->num_sms, st, ws.error);
@@ -419,7 +439,7 @@ hstu_status hstu_stack_forward(hstu_handle* h, const void* values, int64_t T,
   h->last_T = T;
   for (int32_t l = 0; l < num_layers; ++l) {
     const void* x = (l == 0) ? values : out;
-    s = run_layer(h, x, T, ts, &layers[l], out, st);
+    s = run_layer(h, x, T, ts, &layers[l], out, st, l > 0, l + 1 < num_layers);
     if (s != HSTU_OK) return s;
   }
   return HSTU_OK;

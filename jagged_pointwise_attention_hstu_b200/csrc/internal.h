@@ -131,6 +131,9 @@ struct GemmArgs {
   void* out;
   const void* residual;
   int io_fp32;
+  // kBiasResidual with fp32 out only: when set, bf16(out) is written here too
+  // (the next layer's f1 operand), rounded to nearest even
+  void* out_bf16;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error);
 
@@ -180,6 +183,9 @@ bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 // fp32 [outer, inner] row-major, 128-byte swizzle (box_inner * 4 <= 128).
 bool make_tmap_2d_f32_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+// bf16 [outer, inner] row-major, 64-byte swizzle (box_inner * 2 <= 64).
+bool make_tmap_2d_bf16_sw64(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                             uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_1d_i64(CUtensorMap* m, const void* base, uint64_t n, uint32_t box);
 
