@@ -39,19 +39,23 @@
 //   kFast  every key visible to every row of the warp and one time bucket per
 //          row: the whole bias is a per-row constant (plus the position
 //          gather when the position bucket is not clamped);
-//   kMed   every key visible, at most two time buckets per row: one 32-bit
-//          compare of the gap against the row's threshold picks the bias;
+//   kMed   every key visible, at most two time buckets per row: the column
+//          where the row's bucket drops is found once per tile (a binary
+//          search over the tile's sorted key timestamps) and each score
+//          compares its column with it;
 //   kCut   every key visible, at most four time buckets per row: three such
-//          compares and a select chain;
-//   kAny   every key visible to every row, or history rows whose user starts
-//          at or before the tile (the causal diagonal), with gaps below 2^31:
-//          the exact bucket of each gap without a walk -- v = dt + 1 falls in a
-//          bin (floor(log2 v) and the next two bits) spanning less than one
-//          bucket; a per-CTA table gives, per bin, the next bucket's integer
-//          threshold and both candidate biases, so one 16-byte shared load
-//          and one compare give the time bias;
-//   kGen   anything else (user and history boundaries, candidates): the full
-//          mask, position clamp and bucket walk per score.
+//          split columns and a select chain;
+//   kAny   any visibility (the causal diagonal, user and history boundaries,
+//          M-FALCON candidates) with every visible gap of the warp's rows
+//          below 2^31: the full mask per score and the exact bucket of each
+//          gap without a walk -- v = dt + 1 falls in a bin (floor(log2 v) and
+//          the next two bits) spanning less than one bucket; a per-CTA table
+//          gives, per bin, the next bucket's integer threshold and both
+//          candidate biases, so one 16-byte shared load and one compare give
+//          the time bias;
+//   kGen   anything else (the table is not exact for the divisor, or a gap of
+//          2^31 or more): the full mask, position clamp and bucket walk per
+//          score.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -203,7 +207,7 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
     }
     return silu_half(fmaf(acc, 0.5f, add));
   } else if constexpr (MODE == kAny) {
-    const bool vis = jr <= R.i_rel;
+    const bool vis = (unsigned(jr - R.lo_rel) < unsigned(R.hi_rel - R.lo_rel)) || jr == R.i_rel;
     const uint32_t dd = R.ti_lo - uint32_t(tk);     // the gap; < 2^31 - 1 for visible keys
     // masked keys may hold any gap (even -1, i.e. v = 0): keep v >= 1 so the
     // table index stays in [0, 127] for every input
@@ -580,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       R.ti = p.ts[i];
     }
     R.ti_lo = uint32_t(R.ti);
-    const bool history = valid && hi == i + 1 && pos == i;
+    // every visible key of the row lies in its user, at or after ts[lo]: its gap is
+    // at most t_i - ts[lo], so this bound decides whether 32-bit gaps are exact
+    const bool row_narrow = !valid || R.ti - p.ts[lo] < int64_t(0x7FFFFFFE);
     R.b = 0;
     R.cut = R.ti;
     if (valid) {
@@ -619,15 +625,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         walk_to(R.b_last, R.cut_last, kts[127], R.ti, s_thr);
         lev = R.b - R.b_last;
       }
-      const bool narrow = R.ti - kts[0] < int64_t(0x7FFFFFFE);   // gaps fit in int32
       int mode;
       if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
       else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
       else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
       else if (__all_sync(0xffffffffu, full && lev <= 3)) mode = kCut;
-      else if (p.lut_exact &&
-               __all_sync(0xffffffffu, (full || (history && lo <= kb)) && narrow))
-        mode = kAny;
+      else if (p.lut_exact && __all_sync(0xffffffffu, row_narrow))
+        mode = kAny;   // the causal diagonal, user and history boundaries, candidates
       else mode = kGen;
       const bool pc = __all_sync(0xffffffffu, posc);
       if (mode == kFast || mode == kMed || mode == kCut) {
