@@ -194,6 +194,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int c = c_begin; c < c_begin + BN / 2; c += step) {
         const int col0 = nt * BN + c;
+        // fp32 residual: issue its loads first, so that they overlap the
+        // tensor-memory read and the bias adds
+        float4 xres[8];
+        if (!out_bf16) {
+          const float4* res = reinterpret_cast<const float4*>(
+              static_cast<const float*>(p.residual) + grow * int64_t(p.N) + col0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xres[e] = valid ? res[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         float v[64];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -219,11 +228,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              pack_bf16x2(silu_f(v[8 * e + 4]), silu_f(v[8 * e + 5])),
                              pack_bf16x2(silu_f(v[8 * e + 6]), silu_f(v[8 * e + 7])));
         } else if (p.io_fp32) {
-          const float4* res = reinterpret_cast<const float4*>(
-              static_cast<const float*>(p.residual) + grow * int64_t(p.N) + col0);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float4 x = valid ? res[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 x = xres[e];
             v[4 * e + 0] += x.x;
             v[4 * e + 1] += x.y;
             v[4 * e + 2] += x.z;
