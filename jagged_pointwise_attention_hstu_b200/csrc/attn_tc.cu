@@ -549,14 +549,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
-    for (int k = threadIdx.x - 128; k <= clamp + 2 * kPosPad; k += 256)
-      s_rab_pos[k] = p.rab_pos[min(max(k - kPosPad, 0), clamp)];
-    for (int k = threadIdx.x - 128; k < nb; k += 256) {
-      s_rab_time[k] = p.rab_time[k];
-      s_thr[k] = p.thresholds[k];
+    {
+      // the tables, eight global loads in flight per thread before the stores
+      const int t = threadIdx.x - 128;
+      const int n_rp = clamp + 1 + 2 * kPosPad;
+#pragma unroll 1
+      for (int k0 = t; k0 < n_rp; k0 += 8 * 256) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int k = k0 + u * 256;
+          v[u] = k < n_rp ? __ldg(p.rab_pos + min(max(k - kPosPad, 0), clamp)) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (k0 + u * 256 < n_rp) s_rab_pos[k0 + u * 256] = v[u];
+      }
+      const float rt = t < nb ? __ldg(p.rab_time + t) : 0.0f;
+      const int64_t th = t < nb ? __ldg(p.thresholds + t) : 0;
+      const int32_t t32a = __ldg(p.thr32 + t);
+      const int32_t t32b = t + 256 < 257 ? __ldg(p.thr32 + t + 256) : 0;
+      const uint8_t lu = t < 128 ? __ldg(p.time_lut + t) : 0;
+      if (t < nb) {
+        s_rab_time[t] = rt;
+        s_thr[t] = th;
+      }
+      s_thr32[t] = t32a;
+      if (t + 256 < 257) s_thr32[t + 256] = t32b;
+      if (t < 128) s_lut[t] = lu;
     }
-    for (int k = threadIdx.x - 128; k < 257; k += 256) s_thr32[k] = p.thr32[k];
-    if (threadIdx.x - 128 < 128) s_lut[threadIdx.x - 128] = p.time_lut[threadIdx.x - 128];
     named_bar_sync(1, 256);
     if (threadIdx.x - 128 < 128) {
       // per bin: {threshold of the next bucket, bias of the bin's bucket, bias of the next, bucket}
