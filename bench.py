@@ -215,10 +215,15 @@ def attention_traffic(kernel_src_hash, workload_index):
 
 
 def source_hash():
+    """Hash of the attention kernel's code: its source files without comments
+    and blank lines, so that a measurement stays attached to unchanged code."""
     h = hashlib.sha256()
     for name in ("attn_tc.cu", "sm100.cuh"):
-        with open(os.path.join(ROOT, "jagged_pointwise_attention_hstu_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "jagged_pointwise_attention_hstu_b200", "csrc", name)) as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

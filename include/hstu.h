@@ -163,7 +163,7 @@ hstu_status hstu_time_bucket_thresholds(double time_log_div, int32_t num_buckets
 /* ---- Kernel timing (CUDA events on the launching stream) ----
  * When enabled, every kernel the handle launches is bracketed by a pair of
  * CUDA events recorded on the call's stream; the pairs are read back by
- * hstu_get_kernel_timing.  Kinds: 0 schedule (row facts + q-tile order),
+ * hstu_get_kernel_timing.  Kinds: 0 schedule (row facts + work order),
  * 1 fp32->bf16 cast of X, 2 f1 GEMM, 3 attention, 4 LayerNorm-gate, 5 f2 GEMM.
  * At most 4096 launches are recorded between resets. */
 #define HSTU_KERNEL_KINDS 6

@@ -9,20 +9,24 @@
 //
 // One CTA computes one work item -- a pair of adjacent 128-query tiles and
 // one head -- with 12 warps:
-//   warp 0      TMA: both Q tiles once, then K tiles into an NSK-stage ring
-//   warp 1      MMA issue: S_q = Q_q K_j^T into tensor-memory score buffer q
-//               (SS form, both operands K-major in shared memory) and
-//               O_q += P_q V_j with P_q read back from tensor memory (TS form,
-//               V consumed N-major straight from its row-major tile)
-//   warp 2      TMA: V tiles and the keys' timestamps into an NSV-stage ring
+//   warp 0      TMA: both Q tiles once, then K tiles into an NSK-stage ring and
+//               the tiles' key timestamps into a 4-stage ring
+//   warp 1      MMA issue for query tile 0, warp 3 for query tile 1:
+//               S_q = Q_q K_j^T into tensor-memory score buffer q (SS form, both
+//               operands K-major in shared memory) and O_q += P_q V_j with P_q
+//               read back from tensor memory (TS form, V consumed N-major
+//               straight from its row-major tile).  Two issuing threads keep the
+//               tensor pipe fed while either one waits for its row group.
+//   warp 2      TMA: V tiles into an NSV-stage ring
 //   warps 4-7   row group 0: one row of query tile 0 per thread
 //   warps 8-11  row group 1: one row of query tile 1 per thread
 // A row group reads S_q from tensor memory, adds the position and time
 // biases, applies the mask and SiLU and writes P_q (bf16) over the first half
-// of S_q's columns.  The MMAs ping-pong between the query tiles -- while group
-// 0 scores key tile j, the tensor cores run S_1 = Q_1 K_j^T and P_0 V_{j-1} --
-// and every K and V tile loaded feeds both query tiles, which halves the K/V
-// traffic per flop.
+// of S_q's columns.  While one group scores key tile j, the tensor cores run
+// the other group's products, and every K and V tile loaded feeds both query
+// tiles, which halves the K/V traffic per flop.  At the end each group scales
+// its O_q by 1/n_norm, stages it in Q_q's (now free) shared buffer and writes
+// it with TMA stores.
 //
 // Key tiles: only tiles that hold a visible key for some row of the query
 // tile are visited (see sched.cu); the last one is always the diagonal tile.
