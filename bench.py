@@ -214,13 +214,19 @@ def attention_traffic(kernel_src_hash, workload_index):
     return ent.get("dram_bytes_per_launch")
 
 
+HOST_MARKER = "// ==== host side:"
+
+
 def source_hash():
-    """Hash of the attention kernel's code: its source files without comments
-    and blank lines, so that a measurement stays attached to unchanged code."""
+    """Hash of the attention kernel's device code: attn_tc.cu up to its
+    host-side marker line, and sm100.cuh, both without comments and blank
+    lines, so that a measurement stays attached to unchanged device code."""
     h = hashlib.sha256()
     for name in ("attn_tc.cu", "sm100.cuh"):
         with open(os.path.join(ROOT, "jagged_pointwise_attention_hstu_b200", "csrc", name)) as f:
             for line in f:
+                if line.startswith(HOST_MARKER):
+                    break
                 code = line.split("//", 1)[0].rstrip()
                 if code:
                     h.update(code.encode() + b"\n")

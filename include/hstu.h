@@ -91,7 +91,7 @@ typedef struct {
   int32_t time_buckets;     /* rows of rab_time; 1..256 */
   double time_log_div;      /* divisor of ln(1 + dt); > 0 */
   float ln_eps;             /* LayerNorm epsilon (biased variance) */
-  int64_t max_tokens;       /* workspace sizing: largest T of any call; < 2^31 */
+  int64_t max_tokens;       /* workspace sizing: largest T of any call; <= 2^30 */
   int32_t max_users;        /* workspace sizing: largest B of any call */
 } hstu_config;
 

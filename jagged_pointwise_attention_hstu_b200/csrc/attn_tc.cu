@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(1, 256);
     const uint8_t* s_anyb = reinterpret_cast<const uint8_t*>(s_any);
 
-    // token indices fit in int32 (T < 2^31)
+    // token indices fit in int32 (T <= 2^30, checked at create)
     const int i = (qt0 + q) * 128 + row;
     const bool valid = q < nq && i < p.T;
     int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
@@ -788,6 +788,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ==== host side: launch configuration (no device code below this line) ====
+
 template <int HD, bool RECORD>
 cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   using L = AttnLayout<HD>;
@@ -798,14 +800,10 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   if (!make_tmap_1d_i64(&tm_ts, a.ts, uint64_t(a.T), 128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d_f32_sw128(&tm_o, a.av, uint64_t(a.d), uint64_t(a.T), uint64_t(a.d) * 4, 32, 32))
     return cudaErrorInvalidValue;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, RECORD>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(L::smem_bytes(kMaxPosEntries - 1)));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = smem_opt_in(attn_tc_kernel<HD, RECORD>,
+                                    int(L::smem_bytes(kMaxPosEntries - 1)), smem_set);
+  if (e != cudaSuccess) return e;
   AttnParams p;
   p.rows = a.rows;
   p.order = a.order;

@@ -317,14 +317,9 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   if (copy && !make_tmap_2d_bf16_sw64(&to2, a.out_bf16, uint64_t(a.N), uint64_t(a.M),
                                       uint64_t(a.N) * 2, 32, 32))
     return cudaErrorInvalidValue;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(L::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = smem_opt_in(gemm_tc_kernel<BN>, int(L::kSmemBytes), smem_set);
+  if (e != cudaSuccess) return e;
   GemmParams p;
   p.M = a.M;
   p.N = a.N;

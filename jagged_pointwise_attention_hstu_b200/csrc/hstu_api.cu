@@ -174,7 +174,7 @@ hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** ou
     return HSTU_ERR_INVALID_ARG;
   if (c.pos_buckets < 1 || c.pos_clamp < 0 || c.pos_clamp >= c.pos_buckets) return HSTU_ERR_INVALID_ARG;
   if (c.time_buckets < 1 || c.time_buckets > 256 || !(c.time_log_div > 0.0)) return HSTU_ERR_INVALID_ARG;
-  if (!(c.ln_eps >= 0.0f) || c.max_tokens < 0 || c.max_tokens >= (int64_t(1) << 31) ||
+  if (!(c.ln_eps >= 0.0f) || c.max_tokens < 0 || c.max_tokens > hstu::kMaxTokensLimit ||
       c.max_users < 0)
     return HSTU_ERR_INVALID_ARG;
   if (c.pos_clamp > 4096) return HSTU_ERR_UNSUPPORTED;

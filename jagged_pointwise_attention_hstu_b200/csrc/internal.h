@@ -5,12 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/hstu.h"
 
 namespace hstu {
 
 constexpr int kTile = 128;            // query / key rows per attention tile, GEMM BM
 constexpr int64_t kMaxTimestamp = int64_t(1) << 62;
+// Largest max_tokens a handle accepts: the attention kernels index rows with
+// 32-bit integers and round query tiles up past T, so T stays well below 2^31.
+constexpr int64_t kMaxTokensLimit = int64_t(1) << 30;
 
 // Per-token facts the attention kernels need, built by the scheduler.
 //   lo: first row of the token's user; hi: one past the last key the token may
@@ -177,6 +182,23 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st);
 
 // umma_check.cu
 cudaError_t run_umma_tile(int mode, const void* a, const void* b, float* c, int n, int k);
+
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device, once per device: the attribute lives in each device's context, so a
+// process that launches on several GPUs must set it on every one of them.
+// `done` holds one bit per device below 64 (devices above are set every call);
+// two threads racing on the first call both set it, which is harmless.
+template <typename Kernel>
+cudaError_t smem_opt_in(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? uint64_t(1) << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // tensor maps (hstu_api.cu)
 bool make_tmap_2d_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,

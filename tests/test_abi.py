@@ -64,6 +64,8 @@ def _cfg(**kw):
     (dict(time_buckets=0), hstu.HSTU_ERR_INVALID_ARG),
     (dict(time_log_div=0.0), hstu.HSTU_ERR_INVALID_ARG),
     (dict(max_tokens=2 ** 31), hstu.HSTU_ERR_INVALID_ARG),
+    (dict(max_tokens=2 ** 30 + 1), hstu.HSTU_ERR_INVALID_ARG),  # 32-bit row indices
+    (dict(max_tokens=-1), hstu.HSTU_ERR_INVALID_ARG),
     (dict(io_dtype=7), hstu.HSTU_ERR_INVALID_ARG),
     (dict(compute_dtype=hstu.HSTU_DTYPE_FP32), hstu.HSTU_ERR_UNSUPPORTED),  # fp32 math, bf16 io
     (dict(d=320, H=5), hstu.HSTU_ERR_UNSUPPORTED),
