@@ -12,6 +12,11 @@ scaling, no collective on the data path).  Inputs are resident in HBM when
 the timed region starts; `e2e` repeats the measurement with the inputs copied
 from pinned host memory and the output copied back inside every step.
 
+--serve (with an M-FALCON workload, e.g. --workload 4) times serving against
+the history cache instead: the histories are prefilled once and a step scores
+every candidate in calls of --micro-batch candidates per user; its line reports
+candidates/s beside the plain M-FALCON stack over [history ; candidates].
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (one layer over one user's 4096-token causal
 prefix per step), in the same unit.
@@ -80,6 +85,11 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--serve", action="store_true",
+                    help="M-FALCON serving with the history cache (an M-FALCON workload)")
+    ap.add_argument("--micro-batch", type=int, default=None,
+                    help="--serve: candidates per user in one scoring call (default: the "
+                         "workload's micro-batch)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling aid: draw only the first N layers (default: all of the "
                          "workload's layers; per-layer kernels and their sizes are unchanged)")
@@ -265,10 +275,178 @@ def run_reference(args):
     return 0
 
 
+def _pad_pair(n):
+    return (int(n) + 255) // 256 * 256
+
+
+def run_serving(args):
+    """M-FALCON serving against a history cache, on one GPU.  The histories are
+    prefilled once; one step scores every candidate of the batch, in calls of
+    at most `micro_batch` candidates per user.  The same candidates scored by
+    the plain M-FALCON stack over [history ; candidates] are timed beside it."""
+    import torch
+    from jagged_pointwise_attention_hstu_b200 import hstu, runtime
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--serve runs on one GPU")
+    w = wl.WORKLOADS[args.workload]
+    if w.mask != "mfalcon":
+        raise SystemExit("--serve needs an M-FALCON workload")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    batch = wl.make_batch(w, num_layers=args.layers)
+    L = len(batch.layers)
+    B = batch.num_users
+    n_c = [int(c) for c in batch.num_candidates]
+    n_h = [int(n) - c for n, c in zip(batch.lengths, n_c)]
+    offs = [int(o) for o in batch.seq_offsets]
+    hist = np.concatenate([np.arange(offs[b], offs[b] + n_h[b]) for b in range(B)]).astype(np.int64)
+    T_h = len(hist)
+    bm_main = args.micro_batch or w.micro_batch
+    sweep = sorted({bm_main, max(n_c)})
+
+    def make_calls(bm):
+        calls = []   # per call: (packed rows, counts)
+        for k in range(max((c + bm - 1) // bm for c in n_c)):
+            counts = [max(0, min(bm, c - k * bm)) for c in n_c]
+            rows = np.concatenate([np.arange(offs[b] + n_h[b] + k * bm,
+                                             offs[b] + n_h[b] + k * bm + counts[b])
+                                   for b in range(B)])
+            calls.append((rows.astype(np.int64), counts))
+        return calls
+
+    calls_of = {bm: make_calls(bm) for bm in sweep}
+    max_cand_rows = max(sum(_pad_pair(c) for c in counts)
+                        for calls in calls_of.values() for _, counts in calls)
+    rows_cap = _pad_pair(T_h) + max_cand_rows
+    cfg = runtime.config_for(w, max(rows_cap, batch.total_tokens), B)
+    handle = runtime.Handle(cfg, 0)
+    db = runtime.to_device(batch, w.storage, w.compute, dev)
+    structs = [l.struct() for l in db.layers]
+    stream = torch.cuda.current_stream(dev)
+    hidx = torch.from_numpy(hist).to(dev)
+    x_h = db.x[hidx].contiguous()
+    ts_h = db.timestamps[hidx].contiguous()
+    off_h = torch.from_numpy(wl.offsets_from_lengths(np.asarray(n_h)).astype(np.int32)).to(dev)
+    y_h = torch.empty_like(x_h)
+    cache = hstu.hstu_cache_create(handle.h, L, T_h, max_cand_rows)
+    out_full = torch.empty_like(db.x)
+    mode = hstu.HSTU_MASK_MFALCON
+
+    def prefill():
+        hstu.hstu_cache_prefill(handle.h, cache, x_h, T_h, off_h, B, ts_h, structs, y_h, stream)
+
+    def plain_step():
+        hstu.hstu_stack_forward(handle.h, db.x, batch.total_tokens, db.seq_offsets, B,
+                                db.timestamps, structs, mode, db.num_candidates, out_full, stream)
+
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, steps):
+        """Mean device time of `fn`, each run after a 256 MB write (cold L2)."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for s0, s1 in evs:
+            flush.fill_(1)
+            s0.record(stream)
+            fn()
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(s0.elapsed_time(s1) for s0, s1 in evs) / steps
+
+    prefill()
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    results = {}
+    worst = 0.0
+    with ClockSampler(gpu_id) as clk:
+        for _ in range(max(args.warmup, 0)):
+            plain_step()
+        ms_plain = timed(plain_step, args.steps)
+        ms_prefill = timed(prefill, max(1, min(args.steps, 5)))
+        for bm in sweep:
+            inputs = []
+            for rows, counts in calls_of[bm]:
+                ridx = torch.from_numpy(rows).to(dev)
+                inputs.append((db.x[ridx].contiguous(), db.timestamps[ridx].contiguous(), counts))
+            outs = [torch.empty_like(xc) for xc, _, _ in inputs]
+
+            def cached_step():
+                for (xc, tc, counts), yc in zip(inputs, outs):
+                    hstu.hstu_cache_score(handle.h, cache, xc, counts, tc, structs, yc, stream)
+
+            for _ in range(max(args.warmup, 0)):
+                cached_step()
+            torch.cuda.synchronize(dev)
+            hstu.hstu_set_kernel_timing(handle.h, True)
+            ms = timed(cached_step, args.steps)
+            kt = hstu.hstu_get_kernel_timing(handle.h)
+            hstu.hstu_set_kernel_timing(handle.h, False)
+            results[bm] = (ms, kt, len(inputs))
+            # the cached result against the plain stack's candidate rows
+            for (rows, _), yc in zip(calls_of[bm], outs):
+                ref = out_full[torch.from_numpy(rows).to(dev)].double()
+                worst = max(worst, float((yc.double() - ref).abs().max()))
+    if handle.device_error():
+        raise RuntimeError("device error during the timed region")
+    ms, ktimes, n_calls = results[bm_main]
+    bm = bm_main
+    rms = float(out_full.double().pow(2).mean().sqrt())
+    cands = sum(n_c)
+    pairs = sum(c * (h + 1) for c, h in zip(n_c, n_h))
+    attn_flops = 4 * w.head_dim * w.num_heads * pairs * L          # per step
+    pk, pk_kind = peaks()
+    peak_b = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    def attn_tflops(kt):
+        a_ms, a_n = kt["attention"]
+        return attn_flops / (a_ms / args.steps / 1e3) / 1e12 if a_n else None
+
+    achieved = attn_tflops(ktimes)
+    per_step_attn_ms = ktimes["attention"][0] / args.steps
+    # each "block" bracket of a call: rows + order + copy in, then copy out
+    launches = (sum(v[1] for k, v in ktimes.items() if k != "block")
+                + 2 * ktimes["block"][1]) / args.steps
+    by_bm = {str(b): {"value": cands / (m / 1e3), "ms_per_step": m, "calls_per_step": nc,
+                      "attention_tflops": attn_tflops(kt)}
+             for b, (m, kt, nc) in results.items()}
+    line = {
+        "metric": "M-FALCON candidates scored per second against a history cache",
+        "value": cands / (ms / 1e3), "unit": "candidates/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "users": B, "history_tokens": n_h, "candidates": n_c,
+                   "micro_batch": bm, "calls_per_step": n_calls, "layers": L,
+                   "d_model": w.d_model, "heads": w.num_heads, "head_dim": w.head_dim,
+                   "l2": "each step timed alone after a 256 MB write"},
+        "plain_mfalcon_stack": {"value": cands / (ms_plain / 1e3), "unit": "candidates/s",
+                                "ms_per_step": ms_plain,
+                                "note": "hstu_stack_forward over [history ; candidates]"},
+        "by_micro_batch": by_bm,
+        "prefill_ms": ms_prefill,
+        "max_abs_diff_vs_plain": worst, "rms_plain": rms,
+        "roofline": {"bound": "tensor", "kernel": "attention (fused jagged pointwise, tcgen05)",
+                     "achieved": achieved, "peak": peak_b, "unit": "TFLOP/s",
+                     "frac": achieved / peak_b if achieved else None,
+                     "peak_kind": f"{pk_kind} bf16_tflops (burst: short steps)",
+                     "traffic": None, "algorithmic_flops_per_step": attn_flops,
+                     "attention_ms_per_step": per_step_attn_ms},
+        "kernels": {k: {"total_ms": v[0], "launches": v[1]} for k, v in ktimes.items()},
+        "gpu_launches": int(round(launches)),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    hstu.hstu_cache_destroy(cache)
+    handle.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.serve:
+        return run_serving(args)
 
     import torch
     import torch.distributed as dist

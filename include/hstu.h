@@ -164,9 +164,10 @@ hstu_status hstu_time_bucket_thresholds(double time_log_div, int32_t num_buckets
  * When enabled, every kernel the handle launches is bracketed by a pair of
  * CUDA events recorded on the call's stream; the pairs are read back by
  * hstu_get_kernel_timing.  Kinds: 0 schedule (row facts + work order),
- * 1 fp32->bf16 cast of X, 2 f1 GEMM, 3 attention, 4 LayerNorm-gate, 5 f2 GEMM.
+ * 1 fp32->bf16 cast of X, 2 f1 GEMM, 3 attention, 4 LayerNorm-gate, 5 f2 GEMM,
+ * 6 candidate block of a history-cache call (row facts, order, row copies).
  * At most 4096 launches are recorded between resets. */
-#define HSTU_KERNEL_KINDS 6
+#define HSTU_KERNEL_KINDS 7
 
 /* Enables (1) or disables (0) the event pairs; enabling also resets them. */
 hstu_status hstu_set_kernel_timing(hstu_handle* h, int32_t enabled);
@@ -220,6 +221,72 @@ hstu_status hstu_attention_noalloc(const hstu_config* cfg, const void* uvqk, int
                                    const int32_t* num_candidates, const float* rab_pos,
                                    const float* rab_time, float* av, int32_t* device_error,
                                    void* stream);
+
+/* ---- M-FALCON serving with a history cache ----
+ * M-FALCON ranks a user's candidates against the user's history, and the
+ * history's computation does not depend on the candidates (ltzyclt blog on
+ * HSTU, section 5.2, "M-FALCON"; blog "Generative Recommendation 16", item 3:
+ * the candidate-independent history computation is cached).  A cache holds,
+ * for every layer of a stack, SiLU(f1(.)) of the history rows -- the keys and
+ * values a candidate attends to -- plus the history timestamps and offsets.
+ * hstu_cache_prefill runs the stack over the histories once (a causal batch);
+ * each hstu_cache_score call then runs the stack over one micro-batch of
+ * candidates only.  Candidate row outputs are those of hstu_stack_forward in
+ * HSTU_MASK_MFALCON mode on the packed batch [history_b ; candidates_b] per
+ * user: every candidate takes position n_h and sees the history and itself,
+ * so the result of a candidate does not depend on which other candidates
+ * share its call.  The n_norm of the handle must be fixed (> 0).
+ * Inside a call every user's candidates are padded to a multiple of 256 rows
+ * (one pair of 128-row query tiles), so counts that are multiples of 256
+ * waste no work.
+ * Memory of a cache: num_layers * rows_cap * 4d bf16 with
+ * rows_cap = round_up(max_history_tokens, 256) + round_up(max_candidate_rows, 256),
+ * plus a [round_up(max_candidate_rows, 256), d] io_dtype residual block.
+ * A cache belongs to the handle it was created with and uses that handle's
+ * workspace (rows_cap <= max_tokens); calls on one handle or one cache must
+ * not overlap in execution (serialise them on one stream). */
+typedef struct hstu_history_cache_s hstu_history_cache;
+
+/* Allocates (and zeroes) a cache for `num_layers` layers.  Synchronous.
+ *   max_history_tokens  largest T_h of any prefill (>= 0)
+ *   max_candidate_rows  largest padded candidate count of any call, i.e. the sum
+ *                       over users of round_up(n_c, 256); <= 2^21
+ * HSTU_ERR_UNSUPPORTED: compute dtype FP32 or n_norm <= 0;
+ * HSTU_ERR_WORKSPACE: rows_cap above the handle's max_tokens. */
+hstu_status hstu_cache_create(hstu_handle* h, int32_t num_layers, int64_t max_history_tokens,
+                              int64_t max_candidate_rows, hstu_history_cache** out);
+
+/* Frees the cache (synchronizes its device first).  NULL is a no-op. */
+hstu_status hstu_cache_destroy(hstu_history_cache* c);
+
+/* Runs the stack over the histories (causal mode) and keeps each layer's
+ * SiLU(f1(.)) of the history rows, the timestamps and the offsets.  Arguments
+ * as for hstu_stack_forward with HSTU_MASK_CAUSAL; total_tokens <= the
+ * cache's max_history_tokens (else HSTU_ERR_WORKSPACE); num_layers equals the
+ * cache's.  `out` receives the histories' outputs (device [T_h, d] io_dtype,
+ * may alias `values`).  Replaces any earlier history of the cache. */
+hstu_status hstu_cache_prefill(hstu_handle* h, hstu_history_cache* c, const void* values,
+                               int64_t total_tokens, const int32_t* seq_offsets,
+                               int32_t num_users, const int64_t* timestamps,
+                               const hstu_layer_weights* layers, int32_t num_layers, void* out,
+                               void* stream);
+
+/* Scores one micro-batch of candidates against the cached histories.
+ *   values               device [T_c, d] io_dtype: the candidates' layer input,
+ *                        packed by user in the prefill's user order
+ *   num_candidates_host  HOST int32 [num_users of the prefill]: n_c per user
+ *                        (>= 0; T_c = their sum)
+ *   timestamps           device int64 [T_c] (M-FALCON: a candidate carries the
+ *                        time of its user's last history action)
+ *   layers, num_layers   the prefill's weights
+ *   out                  device [T_c, d] io_dtype; may alias `values`
+ * HSTU_ERR_INVALID_ARG before any prefill; HSTU_ERR_WORKSPACE when the padded
+ * candidate rows exceed max_candidate_rows.  Asynchronous on `stream`; the
+ * host array is read before the call returns. */
+hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* values,
+                             const int32_t* num_candidates_host, const int64_t* timestamps,
+                             const hstu_layer_weights* layers, int32_t num_layers, void* out,
+                             void* stream);
 
 /* ---- Inspection entry points for tests (same library, same kernels) ---- */
 

@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <new>
+#include <vector>
 
 #include "internal.h"
 
@@ -251,7 +252,7 @@ hstu_status hstu_destroy(hstu_handle* h) {
 
 namespace {
 
-enum Kind { kSchedule = 0, kCast = 1, kF1 = 2, kAttention = 3, kLnGate = 4, kF2 = 5 };
+enum Kind { kSchedule = 0, kCast = 1, kF1 = 2, kAttention = 3, kLnGate = 4, kF2 = 5, kBlock = 6 };
 
 // Brackets one launch with a pair of events when the handle's timer is on.
 struct Timed {
@@ -296,10 +297,35 @@ hstu_status check_weights(const hstu_layer_weights* w) {
   return HSTU_OK;
 }
 
-// One layer after the schedule is built: f1 -> attention -> LN (.) U -> f2.
+// Where the rows of one layer live.  A plain forward: every row of [0, T) is a
+// query and SiLU(f1(X)) goes to the workspace.  A history-cache call: the
+// buffer is a cache layer's, the layer computes rows [q0, q0 + M) and their
+// attention reads keys anywhere in [0, T_attn).
+struct LayerRows {
+  void* uvqk;              // [T_attn, 4d] compute dtype
+  int64_t q0, M, T_attn;
+  int num_pairs;           // query-tile pairs listed in `order`
+  const int32_t* order;
+  const int64_t* ts;       // [T_attn]
+};
+
+LayerRows plain_rows(hstu_handle* h, int64_t T, const int64_t* ts) {
+  LayerRows r;
+  r.uvqk = h->ws.uvqk;
+  r.q0 = 0;
+  r.M = T;
+  r.T_attn = T;
+  r.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
+  r.order = h->ws.qtile_order;
+  r.ts = ts;
+  return r;
+}
+
+// One layer after the schedule is built: f1 -> attention -> LN (.) U -> f2, on
+// the M query rows; x and out are [M, d].
 // xb_ready: ws.xb already holds bf16(x) (written by the previous layer's f2);
 // make_xb: f2 also writes bf16(out) to ws.xb for the next layer (fp32 io only).
-hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* ts,
+hstu_status run_layer(hstu_handle* h, const void* x, const LayerRows& R,
                       const hstu_layer_weights* w, void* out, cudaStream_t st, bool xb_ready,
                       bool make_xb) {
   const hstu_config& c = h->cfg;
@@ -307,14 +333,19 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   const int d = c.d_model;
   const bool f32 = c.compute_dtype == HSTU_DTYPE_FP32;
   const bool io32 = c.io_dtype == HSTU_DTYPE_FP32;
+  const int64_t T = R.M;
+  const size_t cs = hstu::elem_size(c.compute_dtype);
+  void* uvqk_q = static_cast<char*>(R.uvqk) + size_t(R.q0) * 4 * d * cs;   // the query rows
+  float* av_q = ws.av + size_t(R.q0) * d;
+  if (f32 && R.q0 != 0) return HSTU_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
   hstu::AttnArgs a;
   memset(&a, 0, sizeof(a));
-  a.uvqk = ws.uvqk;
+  a.uvqk = R.uvqk;
   a.av = ws.av;
   a.rows = ws.rows;
-  a.order = ws.qtile_order;
-  a.ts = ts;
+  a.order = R.order;
+  a.ts = R.ts;
   a.thresholds = ws.thresholds;
   a.time_lut = ws.time_lut;
   a.thr32 = ws.thr32;
@@ -323,14 +354,14 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   a.rab_time = w->rab_time;
   a.counters = ws.counters;
   a.error = ws.error;
-  a.T = T;
+  a.T = R.T_attn;
   a.d = d;
   a.H = c.num_heads;
   a.hd = c.head_dim;
   a.pos_clamp = c.pos_clamp;
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
-  a.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
+  a.num_pairs = R.num_pairs;
   if (f32) {
     {
       Timed tm(h, kF1, st);
@@ -370,7 +401,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   g1.K = d;
   g1.epi = hstu::Epi::kSiluSplit;
   g1.bias = w->b1;
-  g1.out = ws.uvqk;
+  g1.out = uvqk_q;
   g1.residual = nullptr;
   g1.io_fp32 = 0;
   g1.out_bf16 = nullptr;
@@ -384,7 +415,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, int64_t T, const int64_t* t
   }
   if (e == cudaSuccess) {
     Timed tm(h, kLnGate, st);
-    e = hstu::launch_ln_gate(ws.av, ws.uvqk, ws.g, w->ln_gamma, w->ln_beta, T, d, c.ln_eps, 0, st);
+    e = hstu::launch_ln_gate(av_q, uvqk_q, ws.g, w->ln_gamma, w->ln_beta, T, d, c.ln_eps, 0, st);
   }
   hstu::GemmArgs g2;
   g2.a = ws.g;
@@ -439,7 +470,7 @@ hstu_status hstu_stack_forward(hstu_handle* h, const void* values, int64_t T,
   h->last_T = T;
   for (int32_t l = 0; l < num_layers; ++l) {
     const void* x = (l == 0) ? values : out;
-    s = run_layer(h, x, T, ts, &layers[l], out, st, l > 0, l + 1 < num_layers);
+    s = run_layer(h, x, plain_rows(h, T, ts), &layers[l], out, st, l > 0, l + 1 < num_layers);
     if (s != HSTU_OK) return s;
   }
   return HSTU_OK;
@@ -720,3 +751,208 @@ extern "C" hstu_status hstu_attention_noalloc(const hstu_config* cfg, const void
     e = cudaMemcpyAsync(device_error, err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// M-FALCON history cache: the candidate-independent history computation of a
+// stack, kept across calls that score micro-batches of candidates.
+struct hstu_history_cache_s {
+  hstu_handle* h = nullptr;    // the handle whose workspace the calls use
+  int device = 0;
+  int32_t num_layers = 0;
+  int64_t max_hist = 0;        // history rows the buffers hold
+  int64_t cand_cap = 0;        // candidate block rows (a multiple of 2 * 128)
+  int64_t rows_cap = 0;        // round_up(max_hist, 256) + cand_cap
+  int32_t max_users = 0;
+  int64_t T_h = -1;            // -1 until the first prefill
+  int32_t B = 0;
+  std::vector<void*> uvqk;     // per layer: device [rows_cap, 4d] bf16
+  int64_t* ts = nullptr;       // device [rows_cap]
+  int32_t* hoff = nullptr;     // device [max_users + 1]
+  int32_t* table = nullptr;    // device [2 * (max_users + 1)]: blk | coff of the last call
+  int32_t* order = nullptr;    // device [cand_cap / 256]
+  void* xblk = nullptr;        // device [cand_cap, d] io dtype: the block's residual stream
+  std::vector<int32_t> table_host;
+};
+
+namespace {
+
+int64_t round_pair(int64_t n) {
+  const int64_t p = 2 * hstu::kTile;
+  return (n + p - 1) / p * p;
+}
+
+}  // namespace
+
+extern "C" {
+
+hstu_status hstu_cache_destroy(hstu_history_cache* c) {
+  if (c == nullptr) return HSTU_OK;
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  for (void* p : c->uvqk)
+    if (p != nullptr) cudaFree(p);
+  void* ptrs[] = {c->ts, c->hoff, c->table, c->order, c->xblk};
+  for (void* p : ptrs)
+    if (p != nullptr) cudaFree(p);
+  delete c;
+  return HSTU_OK;
+}
+
+hstu_status hstu_cache_create(hstu_handle* h, int32_t num_layers, int64_t max_history_tokens,
+                              int64_t max_candidate_rows, hstu_history_cache** out) {
+  if (out == nullptr) return HSTU_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (h == nullptr || num_layers < 1 || max_history_tokens < 0 || max_candidate_rows < 1)
+    return HSTU_ERR_INVALID_ARG;
+  const hstu_config& cfg = h->cfg;
+  if (cfg.compute_dtype != HSTU_DTYPE_BF16 || cfg.n_norm <= 0) return HSTU_ERR_UNSUPPORTED;
+  const int64_t cand_cap = round_pair(max_candidate_rows);
+  if (cand_cap / (2 * hstu::kTile) > hstu::kMaxCandidatePairs) return HSTU_ERR_UNSUPPORTED;
+  const int64_t rows_cap = round_pair(max_history_tokens) + cand_cap;
+  if (rows_cap > cfg.max_tokens || max_history_tokens > cfg.max_tokens) return HSTU_ERR_WORKSPACE;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  hstu_history_cache* c = new (std::nothrow) hstu_history_cache_s();
+  if (c == nullptr) return HSTU_ERR_CUDA;
+  c->h = h;
+  c->device = h->device;
+  c->num_layers = num_layers;
+  c->max_hist = max_history_tokens;
+  c->cand_cap = cand_cap;
+  c->rows_cap = rows_cap;
+  c->max_users = cfg.max_users;
+  const size_t d = size_t(cfg.d_model);
+  const size_t io = hstu::elem_size(cfg.io_dtype);
+  c->uvqk.assign(size_t(num_layers), nullptr);
+  cudaError_t e = cudaSuccess;
+  // Zeroed once: rows never written (the gap before the candidate block, rows
+  // past a shorter history) must hold finite values, since a key tile that
+  // straddles them is multiplied by zero weights on the tensor cores.
+  for (int32_t l = 0; l < num_layers && e == cudaSuccess; ++l) {
+    e = hstu::alloc(&c->uvqk[l], size_t(rows_cap) * 4 * d * 2);
+    if (e == cudaSuccess) e = cudaMemset(c->uvqk[l], 0, size_t(rows_cap) * 4 * d * 2);
+  }
+  if (e == cudaSuccess) e = hstu::alloc(&c->ts, size_t(rows_cap) * 8);
+  if (e == cudaSuccess) e = cudaMemset(c->ts, 0, size_t(rows_cap) * 8);
+  if (e == cudaSuccess) e = hstu::alloc(&c->hoff, size_t(cfg.max_users + 1) * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&c->table, size_t(2 * (cfg.max_users + 1)) * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&c->order, size_t(cand_cap / (2 * hstu::kTile)) * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&c->xblk, size_t(cand_cap) * d * io);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    hstu_cache_destroy(c);
+    return HSTU_ERR_CUDA;
+  }
+  c->table_host.assign(size_t(2 * (cfg.max_users + 1)), 0);
+  *out = c;
+  return HSTU_OK;
+}
+
+hstu_status hstu_cache_prefill(hstu_handle* h, hstu_history_cache* c, const void* values,
+                               int64_t T_h, const int32_t* offsets, int32_t B,
+                               const int64_t* ts, const hstu_layer_weights* layers,
+                               int32_t num_layers, void* out, void* stream) {
+  if (c == nullptr || h == nullptr || c->h != h) return HSTU_ERR_INVALID_ARG;
+  hstu_status s = check_common(h, values, T_h, offsets, B, ts, HSTU_MASK_CAUSAL, nullptr, out);
+  if (s != HSTU_OK) return s;
+  if (T_h > c->max_hist) return HSTU_ERR_WORKSPACE;
+  if (layers == nullptr || num_layers != c->num_layers) return HSTU_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    s = check_weights(&layers[l]);
+    if (s != HSTU_OK) return s;
+  }
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(c->hoff, offsets, size_t(B + 1) * 4, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess && T_h > 0)
+    e = cudaMemcpyAsync(c->ts, ts, size_t(T_h) * 8, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  c->T_h = -1;   // stays invalid unless every launch below is enqueued
+  if (T_h > 0) {
+    {
+      Timed tm(h, kSchedule, st);
+      if (hstu::launch_schedule(h, T_h, offsets, B, ts, HSTU_MASK_CAUSAL, nullptr, st) !=
+          cudaSuccess)
+        return HSTU_ERR_CUDA;
+    }
+    for (int32_t l = 0; l < num_layers; ++l) {
+      LayerRows R = plain_rows(h, T_h, c->ts);
+      R.uvqk = c->uvqk[l];
+      s = run_layer(h, l == 0 ? values : out, R, &layers[l], out, st, l > 0, l + 1 < num_layers);
+      if (s != HSTU_OK) return s;
+    }
+  }
+  c->T_h = T_h;
+  c->B = B;
+  return HSTU_OK;
+}
+
+hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* values,
+                             const int32_t* num_candidates_host, const int64_t* timestamps,
+                             const hstu_layer_weights* layers, int32_t num_layers, void* out,
+                             void* stream) {
+  if (c == nullptr || h == nullptr || c->h != h) return HSTU_ERR_INVALID_ARG;
+  if (c->T_h < 0) return HSTU_ERR_INVALID_ARG;   // no history yet
+  const int32_t B = c->B;
+  if (B > 0 && num_candidates_host == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (layers == nullptr || num_layers != c->num_layers) return HSTU_ERR_INVALID_ARG;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    hstu_status s = check_weights(&layers[l]);
+    if (s != HSTU_OK) return s;
+  }
+  // the block layout, on the host
+  int32_t* blk = c->table_host.data();
+  int32_t* coff = blk + B + 1;
+  int64_t P = 0, T_c = 0;
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t n = num_candidates_host[b];
+    if (n < 0) return HSTU_ERR_INVALID_ARG;
+    blk[b] = int32_t(P);
+    coff[b] = int32_t(T_c);
+    P += round_pair(n);
+    T_c += n;
+    if (P > c->cand_cap) return HSTU_ERR_WORKSPACE;
+  }
+  blk[B] = int32_t(P);
+  coff[B] = int32_t(T_c);
+  if (T_c == 0) return HSTU_OK;
+  if (values == nullptr || out == nullptr || timestamps == nullptr || !hstu::aligned16(values) ||
+      !hstu::aligned16(out) || !hstu::aligned16(timestamps))
+    return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const hstu_config& cfg = h->cfg;
+  const int64_t row_bytes = int64_t(cfg.d_model) * int64_t(hstu::elem_size(cfg.io_dtype));
+  const int64_t q0 = round_pair(c->T_h);
+  // pageable source: the copy is staged before the call returns, so the host
+  // table may be rewritten by the next call
+  cudaError_t e = cudaMemcpyAsync(c->table, c->table_host.data(), size_t(2 * (B + 1)) * 4,
+                                  cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) {
+    Timed tm(h, kBlock, st);
+    e = hstu::launch_candidate_rows(c->table, c->hoff, B, c->T_h, q0, int32_t(P), timestamps,
+                                    c->ts, h->ws.rows, c->order, st);
+    if (e == cudaSuccess)
+      e = hstu::launch_candidate_copy(c->table, B, int32_t(P), row_bytes, values, c->xblk, true, st);
+  }
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  LayerRows R;
+  R.q0 = q0;
+  R.M = P;
+  R.T_attn = q0 + P;
+  R.num_pairs = int(P / (2 * hstu::kTile));
+  R.order = c->order;
+  R.ts = c->ts;
+  for (int32_t l = 0; l < num_layers; ++l) {
+    R.uvqk = c->uvqk[l];
+    const hstu_status s = run_layer(h, c->xblk, R, &layers[l], c->xblk, st, l > 0,
+                                    l + 1 < num_layers);
+    if (s != HSTU_OK) return s;
+  }
+  {
+    Timed tm(h, kBlock, st);
+    e = hstu::launch_candidate_copy(c->table, B, int32_t(P), row_bytes, c->xblk, out, false, st);
+  }
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -122,6 +122,18 @@ cudaError_t launch_schedule_raw(int64_t T, const int32_t* offsets, int32_t B, co
                                 int32_t* order, int32_t* counters, int32_t* err, cudaStream_t st);
 cudaError_t launch_cast_bf16(const float* x, void* xb, int64_t n, cudaStream_t st);
 
+// serve.cu: the candidate block of a history-cache call.  table = blk[0..B]
+// (padded block starts, relative to the block, multiples of 2 * kTile) followed
+// by coff[0..B] (packed candidate offsets); hoff[0..B]: history offsets.
+constexpr int32_t kMaxCandidatePairs = 8192;   // the pair order is ranked in shared memory
+cudaError_t launch_candidate_rows(const int32_t* table, const int32_t* hoff, int32_t B,
+                                  int64_t T_h, int64_t q0, int32_t P, const int64_t* cand_ts,
+                                  int64_t* ts, RowInfo* rows, int32_t* order, cudaStream_t st);
+// to_block: packed candidate rows [T_c, row_bytes] -> block rows [P, row_bytes],
+// padding rows zeroed; else block -> packed (padding rows dropped).
+cudaError_t launch_candidate_copy(const int32_t* table, int32_t B, int32_t P, int64_t row_bytes,
+                                  const void* src, void* dst, bool to_block, cudaStream_t st);
+
 // gemm_tc.cu
 enum class Epi { kSiluSplit = 0, kBiasResidual = 1 };
 struct GemmArgs {

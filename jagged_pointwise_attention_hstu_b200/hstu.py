@@ -94,6 +94,13 @@ def load() -> ctypes.CDLL:
         "hstu_attention_noalloc": (c_int, [POINTER(hstu_config), c_void_p, c_int64, c_void_p,
                                            c_int32, c_void_p, c_int, c_void_p, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_void_p]),
+        "hstu_cache_create": (c_int, [H, c_int32, c_int64, c_int64, POINTER(c_void_p)]),
+        "hstu_cache_destroy": (c_int, [c_void_p]),
+        "hstu_cache_prefill": (c_int, [H, c_void_p, c_void_p, c_int64, c_void_p, c_int32,
+                                       c_void_p, POINTER(hstu_layer_weights), c_int32, c_void_p,
+                                       c_void_p]),
+        "hstu_cache_score": (c_int, [H, c_void_p, c_void_p, POINTER(c_int32), c_void_p,
+                                     POINTER(hstu_layer_weights), c_int32, c_void_p, c_void_p]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -221,7 +228,38 @@ def hstu_attention_noalloc(cfg: hstu_config, uvqk, total_tokens: int, seq_offset
            "hstu_attention_noalloc")
 
 
-KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2")
+def hstu_cache_create(handle, num_layers: int, max_history_tokens: int,
+                      max_candidate_rows: int) -> c_void_p:
+    c = c_void_p()
+    _check(load().hstu_cache_create(handle, num_layers, max_history_tokens, max_candidate_rows,
+                                    ctypes.byref(c)), "hstu_cache_create")
+    return c
+
+
+def hstu_cache_destroy(cache) -> None:
+    _check(load().hstu_cache_destroy(cache), "hstu_cache_destroy")
+
+
+def hstu_cache_prefill(handle, cache, values, total_tokens: int, seq_offsets, num_users: int,
+                       timestamps, layers: Sequence[hstu_layer_weights], out, stream=None) -> None:
+    arr = (hstu_layer_weights * len(layers))(*layers)
+    _check(load().hstu_cache_prefill(handle, cache, _ptr(values), total_tokens, _ptr(seq_offsets),
+                                     num_users, _ptr(timestamps), arr, len(layers), _ptr(out),
+                                     _stream_ptr(stream)),
+           "hstu_cache_prefill")
+
+
+def hstu_cache_score(handle, cache, values, num_candidates: Sequence[int], timestamps,
+                     layers: Sequence[hstu_layer_weights], out, stream=None) -> None:
+    """num_candidates: host integers, one per user of the prefill."""
+    counts = (c_int32 * max(len(num_candidates), 1))(*[int(n) for n in num_candidates])
+    arr = (hstu_layer_weights * len(layers))(*layers)
+    _check(load().hstu_cache_score(handle, cache, _ptr(values), counts, _ptr(timestamps), arr,
+                                   len(layers), _ptr(out), _stream_ptr(stream)),
+           "hstu_cache_score")
+
+
+KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2", "block")
 
 
 def hstu_set_kernel_timing(handle, enabled: bool) -> None:

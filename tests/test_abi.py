@@ -86,3 +86,12 @@ def test_null_arguments_are_rejected(lib):
     assert lib.hstu_get_device_error(None, None) == hstu.HSTU_ERR_INVALID_ARG
     assert lib.hstu_time_bucket_thresholds(0.301, 0, None) == hstu.HSTU_ERR_INVALID_ARG
     assert lib.hstu_debug_umma_tile(0, None, None, None, 128, 64) == hstu.HSTU_ERR_INVALID_ARG
+    c = ctypes.c_void_p()
+    assert lib.hstu_cache_create(None, 1, 16, 256, ctypes.byref(c)) == hstu.HSTU_ERR_INVALID_ARG
+    assert not c.value
+    assert lib.hstu_cache_create(None, 1, 16, 256, None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_cache_destroy(None) == hstu.HSTU_OK
+    assert lib.hstu_cache_prefill(None, None, None, 0, None, 0, None, ctypes.byref(w), 1, None,
+                                  None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_cache_score(None, None, None, None, None, ctypes.byref(w), 1, None,
+                                None) == hstu.HSTU_ERR_INVALID_ARG
