@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the HSTU layer forward (test infrastructure only).
+"""fp64 CPU oracle of the HSTU layer forward and of Stochastic Length sampling
+(test infrastructure only).
 
 Imported only by the tests, the package smoke check and the benchmark's CPU
 baseline leg; the CUDA library shares no code with it.
@@ -7,7 +8,8 @@ from .hstu_oracle import (CAUSAL, MFALCON, OracleConfig, effective_n_norm, f1_sp
                           hstu_layer, hstu_stack, layer_norm, pointwise_attention,
                           position_bucket, silu, time_bucket, user_visibility,
                           visible_pairs)
+from .stochastic_length import keep_whole, stochastic_length
 
 __all__ = ["CAUSAL", "MFALCON", "OracleConfig", "effective_n_norm", "f1_split", "hstu_layer",
            "hstu_stack", "layer_norm", "pointwise_attention", "position_bucket", "silu",
-           "time_bucket", "user_visibility", "visible_pairs"]
+           "time_bucket", "user_visibility", "visible_pairs", "keep_whole", "stochastic_length"]
