@@ -90,6 +90,9 @@ def parse():
     ap.add_argument("--micro-batch", type=int, default=None,
                     help="--serve: candidates per user in one scoring call (default: the "
                          "workload's micro-batch)")
+    ap.add_argument("--sl", action="store_true",
+                    help="Stochastic Length on the device over the raw lengths of the "
+                         "16-user lognormal workload")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling aid: draw only the first N layers (default: all of the "
                          "workload's layers; per-layer kernels and their sizes are unchanged)")
@@ -441,12 +444,97 @@ def run_serving(args):
     return 0
 
 
+def run_sl(args):
+    """Stochastic Length on the device: one call samples the 16-user lognormal
+    workload's raw batch (before sampling; d 512 bf16 rows) and gathers the
+    kept rows and timestamps.  Memory-bound: the roofline is HBM bandwidth."""
+    import torch
+    from jagged_pointwise_attention_hstu_b200 import hstu
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--sl runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[2]
+    rng = np.random.default_rng(np.random.SeedSequence(wl.SEED_BASE + 2))
+    lengths = wl.draw_lengths(w.lengths, w.num_users, rng)
+    offs = wl.offsets_from_lengths(lengths).astype(np.int32)
+    T, B = int(offs[-1]), int(lengths.shape[0])
+    row_bytes = w.d_model * 2
+    u = rng.random(B)
+    keys = rng.integers(0, 2 ** 32, size=T, dtype=np.uint64).astype(np.uint32)
+    vals = torch.from_numpy(rng.normal(size=(T, w.d_model)).astype(np.float32)).to(
+        dev, torch.bfloat16)
+    ts = torch.from_numpy(np.sort(rng.integers(0, 2 ** 40, size=T)).astype(np.int64)).to(dev)
+    offs_d = torch.from_numpy(offs).to(dev)
+    u_d = torch.from_numpy(u).to(dev)
+    keys_d = torch.from_numpy(keys.view(np.int32).copy()).to(dev)
+    out_offs = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    out_idx = torch.empty(T, dtype=torch.int64, device=dev)
+    out_vals = torch.empty_like(vals)
+    out_ts = torch.empty(T, dtype=torch.int64, device=dev)
+    scratch = torch.empty(hstu.hstu_stochastic_length_scratch_bytes(T, B), dtype=torch.uint8,
+                          device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        hstu.hstu_stochastic_length(offs_d, B, T, u_d, keys_d, wl.SL_NC, wl.SL_ALPHA, vals,
+                                    row_bytes, ts, out_offs, out_idx, out_vals, out_ts, scratch,
+                                    err, stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(err.item()):
+        raise RuntimeError(f"device error bits {int(err.item())}")
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(gpu_id) as clk:
+        for s0, s1 in evs:
+            flush.fill_(1)
+            s0.record(stream)
+            step()
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = sum(s0.elapsed_time(s1) for s0, s1 in evs) / args.steps
+    kept = int(out_offs[-1].item())
+    # algorithmic bytes of one call: keys read and flags written + read for every
+    # action; for every kept action its row read and written, its index written
+    # and read back by the gather, its timestamp read and written
+    algo = T * (4 + 2) + kept * (2 * row_bytes + 16 + 16)
+    pk, pk_kind = peaks()
+    peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = algo / (ms / 1e3) / 1e9
+    line = {
+        "metric": "Stochastic Length batch build on the device (input actions per second)",
+        "value": T / (ms / 1e3), "unit": "actions/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 rows", "data": "synthetic",
+        "config": {"workload": f"{w.num_users} users, lognormal lengths (raw, before sampling)",
+                   "actions": T, "kept": kept, "n_c": wl.SL_NC, "alpha": wl.SL_ALPHA,
+                   "row_bytes": row_bytes,
+                   "l2": "each step timed alone after a 256 MB write"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "peak_kind": f"{pk_kind} hbm_gbs",
+                     "traffic": None, "algorithmic_bytes_per_call": algo},
+        "gpu_launches": 4,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.serve:
         return run_serving(args)
+    if args.sl:
+        return run_sl(args)
 
     import torch
     import torch.distributed as dist

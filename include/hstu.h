@@ -76,6 +76,8 @@ typedef enum { HSTU_MASK_CAUSAL = 0, HSTU_MASK_MFALCON = 1 } hstu_mask_mode;
 #define HSTU_DEVERR_CANDIDATES  0x2  /* num_candidates[b] < 0 or > length of user b */
 #define HSTU_DEVERR_TIMESTAMPS  0x4  /* decreasing inside a user, or outside [0, 2^62) */
 #define HSTU_DEVERR_TIMEOUT     0x8  /* a bounded pipeline wait expired */
+#define HSTU_DEVERR_SL_TOO_LONG 0x10 /* Stochastic Length: a sequence to sub-sample is longer
+                                        than HSTU_SL_MAX_SAMPLED_LEN (it is dropped) */
 
 typedef struct {
   int32_t d_model;          /* d = num_heads * head_dim; BF16 compute: 128, 256, 384, 512, 768
@@ -287,6 +289,49 @@ hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* 
                              const int32_t* num_candidates_host, const int64_t* timestamps,
                              const hstu_layer_weights* layers, int32_t num_layers, void* out,
                              void* stream);
+
+/* ---- Stochastic Length on the device ----
+ * Builds the sampled training batch (ltzyclt blog on HSTU, section 5.1; blog
+ * "Generative Recommendation 16", item 2 "Stochastic Length"): a user's
+ * sequence of n actions is kept whole with probability n_c^alpha / n^2 (capped
+ * at 1), otherwise a sub-sequence of n_c actions is sampled uniformly without
+ * replacement and kept in time order (alpha = 1.6, n_c = 776 keeps length 4096
+ * mostly at 776).  The draws are inputs, so the result is a function of them:
+ *   whole  iff  n <= n_c  or  user_uniform[b] * n^2 < n_c^alpha   (fp64, n^2
+ *          exact, one rounding in the product; n_c^alpha from the host pow)
+ *   else   the n_c actions with the smallest (token_keys[t], position) pairs.
+ * Arguments (device pointers unless marked):
+ *   seq_offsets     int32 [B + 1], 0 = offsets[0] <= ... <= offsets[B] = T
+ *   num_users       B >= 0;  total_tokens  T, 0 <= T < 2^31
+ *   user_uniform    fp64 [B] in [0, 1)
+ *   token_keys      uint32 [T]
+ *   n_c, alpha      n_c >= 1, alpha finite
+ *   values          [T, row_bytes] rows to gather, or NULL (indices only);
+ *                   row_bytes a positive multiple of 16, 16-byte aligned
+ *   timestamps      int64 [T] or NULL
+ *   out_offsets     int32 [B + 1]: offsets of the sampled batch
+ *   out_index       int64 [T]: the first out_offsets[B] entries are the global
+ *                   indices of the kept actions, user after user, in time order
+ *   out_values      [T, row_bytes] (needed when values is not NULL): kept rows
+ *   out_timestamps  int64 [T] or NULL: kept timestamps
+ *   scratch         hstu_stochastic_length_scratch_bytes(T, B) bytes, 256-aligned
+ *   device_error    int32 or NULL: overwritten with this call's HSTU_DEVERR_*
+ *                   bits (OFFSETS for a bad offset table -- such users count as
+ *                   empty; SL_TOO_LONG for a dropped sequence), in stream order
+ * Allocates nothing; asynchronous on `stream`.  Sequences that are sampled must
+ * not be longer than HSTU_SL_MAX_SAMPLED_LEN (the sort runs in shared memory). */
+#define HSTU_SL_MAX_SAMPLED_LEN 8192
+
+size_t hstu_stochastic_length_scratch_bytes(int64_t total_tokens, int32_t num_users);
+
+hstu_status hstu_stochastic_length(const int32_t* seq_offsets, int32_t num_users,
+                                   int64_t total_tokens, const double* user_uniform,
+                                   const uint32_t* token_keys, int32_t n_c, double alpha,
+                                   const void* values, int64_t row_bytes,
+                                   const int64_t* timestamps, int32_t* out_offsets,
+                                   int64_t* out_index, void* out_values,
+                                   int64_t* out_timestamps, void* scratch,
+                                   int32_t* device_error, void* stream);
 
 /* ---- Inspection entry points for tests (same library, same kernels) ---- */
 

@@ -956,3 +956,70 @@ hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Stochastic Length: argument checks and the scratch layout
+//   [0, 256)            error word
+//   [256, 256 + 4B')    kept counts (B' = B rounded up to 64)
+//   then                flags [T]
+namespace {
+
+size_t sl_kept_bytes(int32_t B) { return size_t((int64_t(B) + 63) / 64 * 64) * 4; }
+
+}  // namespace
+
+extern "C" {
+
+size_t hstu_stochastic_length_scratch_bytes(int64_t T, int32_t B) {
+  if (T < 0 || B < 0) return 0;
+  return 256 + sl_kept_bytes(B) + size_t((T + 255) / 256 * 256);
+}
+
+hstu_status hstu_stochastic_length(const int32_t* offsets, int32_t B, int64_t T,
+                                   const double* u, const uint32_t* keys, int32_t n_c,
+                                   double alpha, const void* values, int64_t row_bytes,
+                                   const int64_t* ts, int32_t* out_offsets, int64_t* out_index,
+                                   void* out_values, int64_t* out_ts, void* scratch,
+                                   int32_t* device_error, void* stream) {
+  if (B < 0 || T < 0 || T >= (int64_t(1) << 31) || (B == 0 && T != 0)) return HSTU_ERR_INVALID_ARG;
+  if (n_c < 1 || !isfinite(alpha)) return HSTU_ERR_INVALID_ARG;
+  if (offsets == nullptr || out_offsets == nullptr || scratch == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(scratch) % 256 != 0) return HSTU_ERR_INVALID_ARG;
+  if (T > 0 && (u == nullptr || keys == nullptr || out_index == nullptr)) return HSTU_ERR_INVALID_ARG;
+  if (ts != nullptr && out_ts == nullptr) return HSTU_ERR_INVALID_ARG;
+  if (values != nullptr) {
+    if (out_values == nullptr || row_bytes <= 0 || row_bytes % 16 != 0 ||
+        !hstu::aligned16(values) || !hstu::aligned16(out_values))
+      return HSTU_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  hstu::SlArgs a;
+  a.offs = offsets;
+  a.B = B;
+  a.T = T;
+  a.u = u;
+  a.keys = keys;
+  a.n_c = n_c;
+  a.numerator = pow(double(n_c), alpha);
+  a.values = values;
+  a.row_bytes = row_bytes;
+  a.ts = ts;
+  a.out_offs = out_offsets;
+  a.out_index = out_index;
+  a.out_values = out_values;
+  a.out_ts = ts != nullptr ? out_ts : nullptr;
+  a.err = reinterpret_cast<int32_t*>(base);
+  a.kept = reinterpret_cast<int32_t*>(base + 256);
+  a.flags = base + 256 + sl_kept_bytes(B);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = hstu::launch_stochastic_length(a, sms, st);
+  if (e == cudaSuccess && device_error != nullptr)
+    e = cudaMemcpyAsync(device_error, a.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -134,6 +134,29 @@ cudaError_t launch_candidate_rows(const int32_t* table, const int32_t* hoff, int
 cudaError_t launch_candidate_copy(const int32_t* table, int32_t B, int32_t P, int64_t row_bytes,
                                   const void* src, void* dst, bool to_block, cudaStream_t st);
 
+// sl.cu: Stochastic Length over a jagged batch
+constexpr int32_t kSlMaxLen = HSTU_SL_MAX_SAMPLED_LEN;   // longest sequence that is sub-sampled
+struct SlArgs {
+  const int32_t* offs;        // [B + 1]
+  int32_t B;
+  int64_t T;
+  const double* u;            // [B]
+  const uint32_t* keys;       // [T]
+  int32_t n_c;
+  double numerator;           // n_c^alpha
+  const void* values;         // [T, row_bytes] or null
+  int64_t row_bytes;
+  const int64_t* ts;          // [T] or null
+  int32_t* out_offs;          // [B + 1]
+  int64_t* out_index;         // [T]
+  void* out_values;           // [T, row_bytes] or null
+  int64_t* out_ts;            // [T] or null
+  uint8_t* flags;             // scratch [T]
+  int32_t* kept;              // scratch [B]
+  int32_t* err;               // scratch word, cleared first
+};
+cudaError_t launch_stochastic_length(const SlArgs& a, int num_sms, cudaStream_t st);
+
 // gemm_tc.cu
 enum class Epi { kSiluSplit = 0, kBiasResidual = 1 };
 struct GemmArgs {

@@ -101,6 +101,11 @@ def load() -> ctypes.CDLL:
                                        c_void_p]),
         "hstu_cache_score": (c_int, [H, c_void_p, c_void_p, POINTER(c_int32), c_void_p,
                                      POINTER(hstu_layer_weights), c_int32, c_void_p, c_void_p]),
+        "hstu_stochastic_length_scratch_bytes": (c_size_t, [c_int64, c_int32]),
+        "hstu_stochastic_length": (c_int, [c_void_p, c_int32, c_int64, c_void_p, c_void_p,
+                                           c_int32, c_double, c_void_p, c_int64, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_void_p]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -257,6 +262,27 @@ def hstu_cache_score(handle, cache, values, num_candidates: Sequence[int], times
     _check(load().hstu_cache_score(handle, cache, _ptr(values), counts, _ptr(timestamps), arr,
                                    len(layers), _ptr(out), _stream_ptr(stream)),
            "hstu_cache_score")
+
+
+HSTU_SL_MAX_SAMPLED_LEN = 8192
+HSTU_DEVERR_SL_TOO_LONG = 0x10
+
+
+def hstu_stochastic_length_scratch_bytes(total_tokens: int, num_users: int) -> int:
+    return int(load().hstu_stochastic_length_scratch_bytes(total_tokens, num_users))
+
+
+def hstu_stochastic_length(seq_offsets, num_users: int, total_tokens: int, user_uniform,
+                           token_keys, n_c: int, alpha: float, values, row_bytes: int,
+                           timestamps, out_offsets, out_index, out_values, out_timestamps,
+                           scratch, device_error=None, stream=None) -> None:
+    _check(load().hstu_stochastic_length(_ptr(seq_offsets), num_users, total_tokens,
+                                         _ptr(user_uniform), _ptr(token_keys), n_c, alpha,
+                                         _ptr(values), row_bytes, _ptr(timestamps),
+                                         _ptr(out_offsets), _ptr(out_index), _ptr(out_values),
+                                         _ptr(out_timestamps), _ptr(scratch),
+                                         _ptr(device_error), _stream_ptr(stream)),
+           "hstu_stochastic_length")
 
 
 KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2", "block")

@@ -95,3 +95,29 @@ def test_null_arguments_are_rejected(lib):
                                   None) == hstu.HSTU_ERR_INVALID_ARG
     assert lib.hstu_cache_score(None, None, None, None, None, ctypes.byref(w), 1, None,
                                 None) == hstu.HSTU_ERR_INVALID_ARG
+
+
+def test_stochastic_length_host_checks(lib):
+    """Scratch sizing and argument checks return before touching CUDA."""
+    assert lib.hstu_stochastic_length_scratch_bytes(0, 0) == 256
+    assert lib.hstu_stochastic_length_scratch_bytes(1000, 10) == 256 + 256 + 1024
+    assert lib.hstu_stochastic_length_scratch_bytes(-1, 1) == 0
+    P = 256    # a non-null, 256-aligned stand-in pointer; never dereferenced here
+    bad = [
+        dict(B=-1), dict(T=-1), dict(T=2 ** 31), dict(B=0, T=5), dict(n_c=0),
+        dict(alpha=float("nan")), dict(alpha=float("inf")), dict(offsets=None),
+        dict(out_offsets=None), dict(scratch=None), dict(scratch=P + 16), dict(u=None),
+        dict(keys=None), dict(out_index=None), dict(ts=P, out_ts=None),
+        dict(values=P, out_values=None), dict(values=P, out_values=P, row_bytes=24),
+        dict(values=P, out_values=P, row_bytes=0), dict(values=P + 8, out_values=P),
+    ]
+    for over in bad:
+        a = dict(offsets=P, B=2, T=100, u=P, keys=P, n_c=776, alpha=1.6, values=None,
+                 row_bytes=0, ts=None, out_offsets=P, out_index=P, out_values=None,
+                 out_ts=None, scratch=P, err=None)
+        a.update(over)
+        st = lib.hstu_stochastic_length(a["offsets"], a["B"], a["T"], a["u"], a["keys"], a["n_c"],
+                                        a["alpha"], a["values"], a["row_bytes"], a["ts"],
+                                        a["out_offsets"], a["out_index"], a["out_values"],
+                                        a["out_ts"], a["scratch"], a["err"], None)
+        assert st == hstu.HSTU_ERR_INVALID_ARG, over
