@@ -1,6 +1,7 @@
 """The C-ABI library loads and exports every declared entry point; host-side
 logic (argument checks, the time-bucket threshold table) runs without a GPU."""
 import ctypes
+import os
 
 import numpy as np
 import pytest
@@ -121,3 +122,28 @@ def test_stochastic_length_host_checks(lib):
                                         a["out_offsets"], a["out_index"], a["out_values"],
                                         a["out_ts"], a["scratch"], a["err"], None)
         assert st == hstu.HSTU_ERR_INVALID_ARG, over
+
+
+def test_plain_c_consumer_compiles_links_and_runs(tmp_path):
+    """include/hstu.h is plain C99; a C program links every entry point of
+    libhstu.so and calls the host-only ones."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(hstu.LIB_PATH)
+    exe = str(tmp_path / "abi_consumer")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c", "abi_consumer.c"), "-o", exe,
+                    "-L", libdir, "-lhstu", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+    declared = hstu.declared_symbols()
+    assert out[0] == f"entry_points {len(declared)}"
+    thr = hstu.hstu_time_bucket_thresholds(0.301, 128)
+    assert out[1] == f"thresholds {thr[0]} {thr[1]} {thr[3]} {thr[40]}"
+    assert out[2] == "status HSTU_ERR_WORKSPACE"
+    assert out[3] == f"create {hstu.HSTU_ERR_INVALID_ARG} null"
+    assert out[4] == "sl_scratch 1536"
