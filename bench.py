@@ -42,10 +42,25 @@ METRIC = "HSTU layer fwd tokens/s (jagged) and attention TFLOP/s as % of B200 BF
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def rank_batch(w, rank, num_layers=None):
-    """The users of one rank: rank r draws its own seeded batch of workload w
-    (weak scaling; ranks share no data, so the data path has no collective)."""
-    return wl.make_batch(w, seed_offset=rank, num_layers=num_layers)
+def rank_batch(w, rank, num_layers=None, world=1, shard="draw"):
+    """The users of one rank (weak scaling; ranks share no data, so the data
+    path has no collective).
+    shard "draw": rank r draws its own seeded batch of workload w.
+    shard "lpt":  the global batch is every rank's draw (the weights of draw
+                  0), split over the ranks by whole users, longest processing
+                  time first, so that the slowest rank carries as little as
+                  possible; every rank computes the same split."""
+    if shard == "draw" or world <= 1:
+        return wl.make_batch(w, seed_offset=rank, num_layers=num_layers)
+    if shard != "lpt":
+        raise ValueError(f"unknown shard mode {shard!r}")
+    from jagged_pointwise_attention_hstu_b200 import sharding
+    draws = [wl.make_batch(w, seed_offset=r, num_layers=num_layers if r == 0 else 1)
+             for r in range(world)]
+    glob = sharding.concat_batches(draws)
+    costs = sharding.user_costs(glob.lengths, glob.num_candidates, w.d_model, w.num_heads,
+                                w.head_dim, w.mask == "mfalcon")
+    return sharding.shard_batch(glob, sharding.lpt_shards(costs, world)[rank])
 
 
 def _reduce(x, world, device, op):
@@ -85,6 +100,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--shard", choices=["draw", "lpt"], default="draw",
+                    help="users of each rank: its own seeded draw, or an LPT split of "
+                         "all ranks' draws")
     ap.add_argument("--serve", action="store_true",
                     help="M-FALCON serving with the history cache (an M-FALCON workload)")
     ap.add_argument("--micro-batch", type=int, default=None,
@@ -550,7 +568,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     w = wl.WORKLOADS[args.workload]
-    batch = rank_batch(w, rank, num_layers=args.layers)
+    batch = rank_batch(w, rank, num_layers=args.layers, world=world, shard=args.shard)
     L = len(batch.layers)
     T = batch.total_tokens
     cfg = runtime.config_for(w, T, batch.num_users)
@@ -732,7 +750,8 @@ def main():
         "config": {"workload": w.name, "users_per_gpu": batch.num_users, "tokens_per_gpu": T,
                    "layers": L, "d_model": w.d_model, "heads": w.num_heads,
                    "head_dim": w.head_dim, "residual_stream": w.storage,
-                   "parallelism": f"dp{world} (users sharded, no collective)",
+                   "parallelism": f"dp{world} (users sharded, no collective; "
+                                  f"shard {args.shard})",
                    "l2": l2_note,
                    "unit_note": "tokens/s counts token-layers: tokens x layers / step time"},
         "attention": {"tflops": attn_tflops, "pct_of_sustained_peak": 100 * attn_tflops / peak_s if attn_tflops else None,
