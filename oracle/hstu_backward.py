@@ -26,8 +26,8 @@ from typing import Dict
 
 import numpy as np
 
-from .hstu_oracle import (MFALCON, OracleConfig, effective_n_norm, silu, user_rab,
-                          user_visibility)
+from .hstu_oracle import (MFALCON, OracleConfig, effective_n_norm, pointwise_attention, silu,
+                          user_rab, user_visibility)
 
 
 def sigmoid(x: np.ndarray) -> np.ndarray:
@@ -47,6 +47,53 @@ def _params(params) -> Dict[str, np.ndarray]:
             for k in ("w1", "b1", "w2", "b2", "rab_pos", "rab_time", "ln_gamma", "ln_beta")}
 
 
+def pointwise_attention_backward(Q, K, V, dO, seq_offsets, timestamps, num_candidates,
+                                 rab_pos, rab_time, cfg: OracleConfig):
+    """Gradients of sum(dO * O) for O = pointwise_attention(Q, K, V, ...):
+    returns (dQ, dK, dV, d_rab_pos, d_rab_time).  Per user and head, with
+    s = q.k + rab and a = vis * SiLU(s) / n_norm:
+        dV = a^T dO,  dA = dO V^T,  dS = vis * dA * SiLU'(s) / n_norm,
+        dQ = dS K,    dK = dS^T Q,
+    and each bias entry collects dS of every visible (query, key, head) that
+    reads it."""
+    Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, dO))
+    rab_pos = np.asarray(rab_pos, dtype=np.float64)
+    rab_time = np.asarray(rab_time, dtype=np.float64)
+    H, hd = cfg.num_heads, cfg.head_dim
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    lengths = offs[1:] - offs[:-1]
+    nn = effective_n_norm(cfg, lengths)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    d_pos = np.zeros_like(rab_pos)
+    d_time = np.zeros_like(rab_time)
+    for b in range(len(lengths)):
+        lo, hi = int(offs[b]), int(offs[b + 1])
+        n = hi - lo
+        if n == 0:
+            continue
+        n_c = int(num_candidates[b]) if (num_candidates is not None and cfg.mask == MFALCON) else 0
+        q_local = np.arange(n)
+        vis, rel = user_visibility(n, n_c, cfg.mask, q_local)
+        rab, pidx, tidx = user_rab(np.asarray(timestamps[lo:hi]), q_local, rel, rab_pos,
+                                   rab_time, cfg)
+        d_rab = np.zeros(vis.shape)
+        for h in range(H):
+            c = slice(h * hd, (h + 1) * hd)
+            s = Q[lo:hi, c] @ K[lo:hi, c].T + rab
+            a = np.where(vis, silu(s) / nn, 0.0)
+            dV[lo:hi, c] += a.T @ dO[lo:hi, c]
+            da = dO[lo:hi, c] @ V[lo:hi, c].T
+            ds = np.where(vis, da * silu_grad(s) / nn, 0.0)
+            dQ[lo:hi, c] += ds @ K[lo:hi, c]
+            dK[lo:hi, c] += ds.T @ Q[lo:hi, c]
+            d_rab += ds
+        np.add.at(d_pos, pidx[vis], d_rab[vis])
+        np.add.at(d_time, tidx[vis], d_rab[vis])
+    return dQ, dK, dV, d_pos, d_time
+
+
 def hstu_layer_backward(X, seq_offsets, timestamps, num_candidates, params, cfg: OracleConfig,
                         dY) -> Dict[str, np.ndarray]:
     """Gradients of sum(dY * Y) for Y = hstu_layer(X, ...)["Y"].
@@ -56,34 +103,14 @@ def hstu_layer_backward(X, seq_offsets, timestamps, num_candidates, params, cfg:
     X = np.asarray(X, dtype=np.float64)
     dY = np.asarray(dY, dtype=np.float64)
     p = _params(params)
-    d, H, hd = cfg.d_model, cfg.num_heads, cfg.head_dim
-    offs = np.asarray(seq_offsets, dtype=np.int64)
-    lengths = offs[1:] - offs[:-1]
-    nn = effective_n_norm(cfg, lengths)
+    d = cfg.d_model
 
     # ---- forward, keeping what the backward reads
     H1 = X @ p["w1"].T + p["b1"]                       # equation (1), before phi1
     Z = silu(H1)
     U, V, Q, K = Z[:, :d], Z[:, d:2 * d], Z[:, 2 * d:3 * d], Z[:, 3 * d:]
-    T = X.shape[0]
-    O = np.zeros((T, d))
-    blocks = []                                        # per user: (lo, hi, vis, pidx, tidx, rab)
-    for b in range(len(lengths)):
-        lo, hi = int(offs[b]), int(offs[b + 1])
-        n = hi - lo
-        if n == 0:
-            continue
-        n_c = int(num_candidates[b]) if (num_candidates is not None and cfg.mask == MFALCON) else 0
-        q_local = np.arange(n)
-        vis, rel = user_visibility(n, n_c, cfg.mask, q_local)
-        rab, pidx, tidx = user_rab(np.asarray(timestamps[lo:hi]), q_local, rel, p["rab_pos"],
-                                   p["rab_time"], cfg)
-        blocks.append((lo, hi, vis, pidx, tidx, rab))
-        for h in range(H):
-            c = slice(h * hd, (h + 1) * hd)
-            s = Q[lo:hi, c] @ K[lo:hi, c].T + rab
-            a = np.where(vis, silu(s) / nn, 0.0)
-            O[lo:hi, c] = a @ V[lo:hi, c]
+    O = pointwise_attention(Q, K, V, seq_offsets, timestamps, num_candidates, p["rab_pos"],
+                            p["rab_time"], cfg)
     mu = O.mean(axis=1, keepdims=True)
     var = ((O - mu) ** 2).mean(axis=1, keepdims=True)
     rstd = 1.0 / np.sqrt(var + cfg.ln_eps)
@@ -108,25 +135,8 @@ def hstu_layer_backward(X, seq_offsets, timestamps, num_candidates, params, cfg:
                  - Ohat * (dOhat * Ohat).mean(axis=1, keepdims=True))
 
     # ---- equation (2): O = a V with a = vis * SiLU(Q K^T + rab) / n_norm
-    dQ = np.zeros_like(Q)
-    dK = np.zeros_like(K)
-    dV = np.zeros_like(V)
-    g["rab_pos"] = np.zeros_like(p["rab_pos"])
-    g["rab_time"] = np.zeros_like(p["rab_time"])
-    for lo, hi, vis, pidx, tidx, rab in blocks:
-        d_rab = np.zeros(vis.shape)
-        for h in range(H):
-            c = slice(h * hd, (h + 1) * hd)
-            s = Q[lo:hi, c] @ K[lo:hi, c].T + rab
-            a = np.where(vis, silu(s) / nn, 0.0)
-            dV[lo:hi, c] += a.T @ dO[lo:hi, c]
-            da = dO[lo:hi, c] @ V[lo:hi, c].T
-            ds = np.where(vis, da * silu_grad(s) / nn, 0.0)
-            dQ[lo:hi, c] += ds @ K[lo:hi, c]
-            dK[lo:hi, c] += ds.T @ Q[lo:hi, c]
-            d_rab += ds
-        np.add.at(g["rab_pos"], pidx[vis], d_rab[vis])
-        np.add.at(g["rab_time"], tidx[vis], d_rab[vis])
+    dQ, dK, dV, g["rab_pos"], g["rab_time"] = pointwise_attention_backward(
+        Q, K, V, dO, seq_offsets, timestamps, num_candidates, p["rab_pos"], p["rab_time"], cfg)
 
     # ---- equation (1): Z = SiLU(X W1^T + b1), split U | V | Q | K
     dZ = np.concatenate([dU, dV, dQ, dK], axis=1)
