@@ -333,6 +333,27 @@ hstu_status hstu_stochastic_length(const int32_t* seq_offsets, int32_t num_users
                                    int64_t* out_timestamps, void* scratch,
                                    int32_t* device_error, void* stream);
 
+/* ---- Backward of the attention step ----
+ * Gradients of sum(dO * O) for O of equation (2), computed by the handle's
+ * tensor-core backward kernel: with s = q.k + rab and a = vis SiLU(s) / n_norm,
+ *   dV = a^T dO,  dQ = dS K,  dK = dS^T Q,  dS = vis (dO V^T) SiLU'(s) / n_norm,
+ * and every rab_pos / rab_time entry collects dS of each visible pair and head
+ * reading it.  Builds the jagged schedule from the same arguments as the
+ * forward.
+ *   uvqk            device bf16 [T, 4d]: the forward's SiLU(X W1^T + b1)
+ *   d_out           device bf16 [T, d]: dO
+ *   dq, dk, dv      device fp32 [T, d] (overwritten)
+ *   d_rab_pos       device fp32 [pos_buckets] (overwritten)
+ *   d_rab_time      device fp32 [time_buckets] (overwritten)
+ * Other arguments as for hstu_layer_forward; compute dtype BF16 only. */
+hstu_status hstu_attention_backward(hstu_handle* h, const void* uvqk, const void* d_out,
+                                    int64_t total_tokens, const int32_t* seq_offsets,
+                                    int32_t num_users, const int64_t* timestamps,
+                                    hstu_mask_mode mask_mode, const int32_t* num_candidates,
+                                    const float* rab_pos, const float* rab_time, float* dq,
+                                    float* dk, float* dv, float* d_rab_pos, float* d_rab_time,
+                                    void* stream);
+
 /* ---- Inspection entry points for tests (same library, same kernels) ---- */
 
 typedef enum {

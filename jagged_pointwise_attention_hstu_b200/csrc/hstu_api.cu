@@ -1023,3 +1023,55 @@ hstu_status hstu_stochastic_length(const int32_t* offsets, int32_t B, int64_t T,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward of the attention step
+extern "C" hstu_status hstu_attention_backward(
+    hstu_handle* h, const void* uvqk, const void* d_out, int64_t T, const int32_t* offsets,
+    int32_t B, const int64_t* ts, hstu_mask_mode mode, const int32_t* ncand, const float* rab_pos,
+    const float* rab_time, float* dq, float* dk, float* dv, float* d_rab_pos, float* d_rab_time,
+    void* stream) {
+  hstu_status s = check_common(h, uvqk, T, offsets, B, ts, mode, ncand, d_out);
+  if (s != HSTU_OK) return s;
+  if (h->cfg.compute_dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (T == 0) return HSTU_OK;
+  const void* ps[] = {rab_pos, rab_time, dq, dk, dv, d_rab_pos, d_rab_time};
+  for (const void* q : ps)
+    if (q == nullptr || !hstu::aligned16(q)) return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu_config& c = h->cfg;
+  const size_t d = size_t(c.d_model);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dq, 0, size_t(T) * d * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_pos, 0, size_t(c.pos_buckets) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, size_t(c.time_buckets) * 4, st);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  hstu::AttnBwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.uvqk = uvqk;
+  a.dO = d_out;
+  a.rows = h->ws.rows;
+  a.offsets = offsets;
+  a.B = B;
+  a.ts = ts;
+  a.thresholds = h->ws.thresholds;
+  a.rab_pos = rab_pos;
+  a.rab_time = rab_time;
+  a.counters = h->ws.counters;
+  a.error = h->ws.error;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.d_rab_pos = d_rab_pos;
+  a.d_rab_time = d_rab_time;
+  a.T = T;
+  a.d = c.d_model;
+  a.H = c.num_heads;
+  a.hd = c.head_dim;
+  a.pos_clamp = c.pos_clamp;
+  a.time_buckets = c.time_buckets;
+  a.n_norm_fixed = c.n_norm;
+  e = hstu::launch_attention_bwd_tc(a, st);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}

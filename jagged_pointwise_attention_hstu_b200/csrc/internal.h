@@ -204,6 +204,30 @@ struct AttnArgs {
 };
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t st, bool record);
 
+// attn_bwd_tc.cu: backward of the attention step
+struct AttnBwdArgs {
+  const void* uvqk;          // [T, 4d] bf16 (the forward's U | V | Q | K)
+  const void* dO;            // [T, d] bf16: gradient of the attention output O
+  const RowInfo* rows;       // the forward's row facts
+  const int32_t* offsets;    // [B + 1]
+  int32_t B;
+  const int64_t* ts;
+  const int64_t* thresholds; // [time_buckets]
+  const float* rab_pos;
+  const float* rab_time;
+  const int32_t* counters;   // [0] = n_norm when not fixed
+  int32_t* error;
+  float* dq;                 // [T, d] fp32, zeroed by the caller (accumulated)
+  float* dk;                 // [T, d] fp32 (written)
+  float* dv;                 // [T, d] fp32 (written)
+  float* d_rab_pos;          // [pos_buckets] fp32, zeroed by the caller (accumulated)
+  float* d_rab_time;         // [time_buckets] fp32, zeroed by the caller (accumulated)
+  int64_t T;
+  int d, H, hd;
+  int pos_clamp, time_buckets, n_norm_fixed;
+};
+cudaError_t launch_attention_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
+
 // ln_gate.cu
 cudaError_t launch_ln_gate(const float* av, const void* uvqk, void* g, const float* gamma,
                            const float* beta, int64_t T, int d, float eps, int compute_fp32,

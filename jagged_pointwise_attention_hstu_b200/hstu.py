@@ -106,6 +106,10 @@ def load() -> ctypes.CDLL:
                                            c_int32, c_double, c_void_p, c_int64, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p]),
+        "hstu_attention_backward": (c_int, [H, c_void_p, c_void_p, c_int64, c_void_p, c_int32,
+                                            c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_void_p]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -283,6 +287,17 @@ def hstu_stochastic_length(seq_offsets, num_users: int, total_tokens: int, user_
                                          _ptr(out_timestamps), _ptr(scratch),
                                          _ptr(device_error), _stream_ptr(stream)),
            "hstu_stochastic_length")
+
+
+def hstu_attention_backward(handle, uvqk, d_out, total_tokens: int, seq_offsets, num_users: int,
+                            timestamps, mask_mode: int, num_candidates, rab_pos, rab_time, dq, dk,
+                            dv, d_rab_pos, d_rab_time, stream=None) -> None:
+    _check(load().hstu_attention_backward(handle, _ptr(uvqk), _ptr(d_out), total_tokens,
+                                          _ptr(seq_offsets), num_users, _ptr(timestamps),
+                                          mask_mode, _ptr(num_candidates), _ptr(rab_pos),
+                                          _ptr(rab_time), _ptr(dq), _ptr(dk), _ptr(dv),
+                                          _ptr(d_rab_pos), _ptr(d_rab_time), _stream_ptr(stream)),
+           "hstu_attention_backward")
 
 
 KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2", "block")
