@@ -111,6 +111,8 @@ def parse():
     ap.add_argument("--sl", action="store_true",
                     help="Stochastic Length on the device over the raw lengths of the "
                          "16-user lognormal workload")
+    ap.add_argument("--attn-bwd", action="store_true",
+                    help="time the attention backward on one layer of the workload")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling aid: draw only the first N layers (default: all of the "
                          "workload's layers; per-layer kernels and their sizes are unchanged)")
@@ -545,8 +547,91 @@ def run_sl(args):
     return 0
 
 
+def run_attn_bwd(args):
+    """The attention step's backward on one layer of the workload: U|V|Q|K from
+    a forward of the first layer, a random bf16 dO; the kernel's algorithmic
+    flops are 2.5x the forward's (S recomputed, dA, dV, dK, dQ: 10 hd per
+    visible pair and head)."""
+    import torch
+    from jagged_pointwise_attention_hstu_b200 import hstu, runtime
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--attn-bwd runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.workload]
+    if w.compute != "bf16":
+        raise SystemExit("--attn-bwd needs a bf16 workload")
+    batch = wl.make_batch(w, num_layers=1)
+    T, d = batch.total_tokens, w.d_model
+    cfg = runtime.config_for(w, T, batch.num_users)
+    handle = runtime.Handle(cfg, 0)
+    db = runtime.to_device(batch, w.storage, w.compute, dev)
+    mode = runtime.mask_mode_of(w)
+    y = torch.empty_like(db.x)
+    handle.forward(db, y, mode)
+    uvqk = handle.intermediate(hstu.HSTU_TENSOR_UVQK, T)
+    dO = torch.randn((T, d), generator=torch.Generator(device=dev).manual_seed(3), device=dev,
+                     dtype=torch.float32).to(torch.bfloat16)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty((T, d), **f32) for _ in range(3))
+    g_pos = torch.empty(w.pos_buckets, **f32)
+    g_time = torch.empty(w.time_buckets, **f32)
+    lp = db.layers[0]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        hstu.hstu_attention_backward(handle.h, uvqk, dO, T, db.seq_offsets, db.num_users,
+                                     db.timestamps, mode, db.num_candidates, lp.rab_pos,
+                                     lp.rab_time, dq, dk, dv, g_pos, g_time, stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize(dev)
+    if handle.device_error():
+        raise RuntimeError("device error during warm-up")
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(gpu_id) as clk:
+        for s0, s1 in evs:
+            flush.fill_(1)
+            s0.record(stream)
+            step()
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+    if handle.device_error():
+        raise RuntimeError("device error during the timed region")
+    ms = sum(s0.elapsed_time(s1) for s0, s1 in evs) / args.steps
+    attn_fwd, _ = workload_flops(w, batch)
+    flops = 2.5 * attn_fwd
+    pk, pk_kind = peaks()
+    peak_b = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "attention backward TFLOP/s (dQ, dK, dV and bias-table gradients, one layer)",
+        "value": achieved, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": T, "d_model": d, "heads": w.num_heads,
+                   "head_dim": w.head_dim,
+                   "note": "the step includes the schedule and the zeroing of dQ and the "
+                           "bias gradients; each step timed alone after a 256 MB write"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_b, "unit": "TFLOP/s",
+                     "frac": achieved / peak_b, "peak_kind": f"{pk_kind} bf16_tflops (burst)",
+                     "traffic": None, "algorithmic_flops_per_step": flops},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    handle.close()
+    return 0
+
+
 def main():
     args = parse()
+    if args.attn_bwd:
+        return run_attn_bwd(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.serve:
