@@ -326,7 +326,10 @@ def run_serving(args):
     hist = np.concatenate([np.arange(offs[b], offs[b] + n_h[b]) for b in range(B)]).astype(np.int64)
     T_h = len(hist)
     bm_main = args.micro_batch or w.micro_batch
-    sweep = sorted({bm_main, max(n_c)})
+    # the workload's micro-batch, the whole candidate set in one call, and the
+    # powers of two between 128 and it: calls per step against throughput
+    top = max(n_c)
+    sweep = sorted({bm_main, top} | {b for b in (128, 256, 512, 1024, 2048) if b < top})
 
     def make_calls(bm):
         calls = []   # per call: (packed rows, counts)
