@@ -129,7 +129,7 @@ struct AttnLayout {
   static_assert(kTileBytes % 1024 == 0, "tile stride alignment");
   static_assert(kKts % 128 == 0, "timestamp stage alignment");
   static_assert(kBars % 8 == 0, "mbarrier alignment");
-  // O of query tile q is staged for its TMA stores in Q_q's tile, in two rounds:
+  // O of query tile q is staged for its TMA stores in Q_q's tile, in two passes:
   // per warp a quarter of the tile holds HD / 64 boxes of 32 rows x 32 fp32 columns
   static_assert((kTileBytes / 4) % 4096 == 0 && (kTileBytes / 4) / 4096 == HD / 64, "O staging");
   static_assert(smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         tc_fence_after();
         uint8_t* stage = smem + L::kQ + q * L::kTileBytes + wq * (L::kTileBytes / 4);
-        constexpr int kBoxes = HD / 64;   // boxes per round; two rounds cover HD columns
+        constexpr int kBoxes = HD / 64;   // boxes per pass; two passes cover HD columns
 #pragma unroll 1
         for (int rd = 0; rd < 2; ++rd) {
 #pragma unroll 1
@@ -769,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_store_2d(&tm_o, stage + cb * 4096, h * HD + (rd * kBoxes + cb) * 32,
                            (qt0 + q) * 128 + wq * 32);
             bulk_commit_group();
-            bulk_wait_group_read0();   // the boxes are reused by the next round
+            bulk_wait_group_read0();   // the boxes are reused by the next pass
           }
           __syncwarp();
         }
