@@ -297,6 +297,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!w) { ok = false; break; }
       tc_fence_after();
       bool any = false;
+      // Along a row the keys advance in time inside the user, so the gap only
+      // shrinks: the time bucket walks down from the previous visible key's (a
+      // larger gap, i.e. input out of order, searches again).  The bias
+      // gradients are summed in registers while the bucket stays the same
+      // (time) or for the clamped entry (position), and added to shared
+      // memory when the bucket changes and at the end of the tile.
+      int tb = -1;
+      float acc_t = 0.0f, acc_c = 0.0f;
 #pragma unroll 1
       for (int c0 = 0; c0 < 128; c0 += 32) {
         uint32_t rs[32], ra[32];
@@ -317,15 +325,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (vis) {
               int64_t rel = pos - j;
               const int pidx = rel < 0 ? 0 : (rel > clamp ? clamp : int(rel));
-              const int tidx = bwd_bucket(s_thr, nb, ti - s_kts[c]);
+              const int64_t gap = ti - s_kts[c];
+              int tidx;
+              if (tb < 0 || (tb + 1 < nb && gap >= s_thr[tb + 1])) {
+                tidx = bwd_bucket(s_thr, nb, gap);
+              } else {
+                tidx = tb;
+                while (tidx > 0 && gap < s_thr[tidx]) --tidx;
+              }
               const float s = __uint_as_float(rs[e + f]) + __ldg(p.rab_pos + pidx) +
                               __ldg(p.rab_time + tidx);
               const float sig = 0.5f + 0.5f * tanh_approx(0.5f * s);
               av[f] = s * sig * inv_nn;
               const float ds = __uint_as_float(ra[e + f]) * (sig * (1.0f + s * (1.0f - sig))) * inv_nn;
               dv[f] = ds;
-              atomicAdd(s_gpos + pidx, ds);
-              atomicAdd(s_gtime + tidx, ds);
+              if (pidx == clamp) acc_c += ds;
+              else atomicAdd(s_gpos + pidx, ds);
+              if (tidx != tb) {
+                if (tb >= 0 && acc_t != 0.0f) atomicAdd(s_gtime + tb, acc_t);
+                tb = tidx;
+                acc_t = 0.0f;
+              }
+              acc_t += ds;
               any = true;
             }
           }
@@ -340,6 +361,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           st_shared_v4_u32(smem_u32(sDS + off), pd[4 * g], pd[4 * g + 1], pd[4 * g + 2], pd[4 * g + 3]);
         }
       }
+      if (tb >= 0 && acc_t != 0.0f) atomicAdd(s_gtime + tb, acc_t);
+      if (acc_c != 0.0f) atomicAdd(s_gpos + clamp, acc_c);
       fence_proxy_async_smem();   // the tensor cores read P and dS through the async proxy
       tc_fence_before();
       mbar_arrive(p_full);
