@@ -429,9 +429,8 @@ def run_serving(args):
 
     achieved = attn_tflops(ktimes)
     per_step_attn_ms = ktimes["attention"][0] / args.steps
-    # each "block" bracket of a call: rows + order + copy in, then copy out
-    launches = (sum(v[1] for k, v in ktimes.items() if k != "block")
-                + 2 * ktimes["block"][1]) / args.steps
+    # the "block" brackets of a call: the fused rows + copy-in launch, then the copy-out
+    launches = sum(v[1] for v in ktimes.values()) / args.steps
     by_bm = {str(b): {"value": cands / (m / 1e3), "ms_per_step": m, "calls_per_step": nc,
                       "attention_tflops": attn_tflops(kt)}
              for b, (m, kt, nc) in results.items()}

@@ -284,7 +284,10 @@ hstu_status hstu_cache_prefill(hstu_handle* h, hstu_history_cache* c, const void
  *   out                  device [T_c, d] io_dtype; may alias `values`
  * HSTU_ERR_INVALID_ARG before any prefill; HSTU_ERR_WORKSPACE when the padded
  * candidate rows exceed max_candidate_rows.  Asynchronous on `stream`; the
- * host array is read before the call returns. */
+ * host array is read before the call returns.  The call's layout table and
+ * pair order go to the device from one of four pinned staging slots; a slot
+ * is reused only after its previous copy has finished, and the first call
+ * after a prefill waits for the prefill's copy of the history offsets. */
 hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* values,
                              const int32_t* num_candidates_host, const int64_t* timestamps,
                              const hstu_layer_weights* layers, int32_t num_layers, void* out,

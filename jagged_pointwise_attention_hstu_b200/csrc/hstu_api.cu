@@ -9,7 +9,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "internal.h"
@@ -756,6 +758,7 @@ extern "C" hstu_status hstu_attention_noalloc(const hstu_config* cfg, const void
 // M-FALCON history cache: the candidate-independent history computation of a
 // stack, kept across calls that score micro-batches of candidates.
 struct hstu_history_cache_s {
+  static constexpr int kRing = 4;   // pinned staging slots for the per-call table
   hstu_handle* h = nullptr;    // the handle whose workspace the calls use
   int device = 0;
   int32_t num_layers = 0;
@@ -768,10 +771,16 @@ struct hstu_history_cache_s {
   std::vector<void*> uvqk;     // per layer: device [rows_cap, 4d] bf16
   int64_t* ts = nullptr;       // device [rows_cap]
   int32_t* hoff = nullptr;     // device [max_users + 1]
-  int32_t* table = nullptr;    // device [2 * (max_users + 1)]: blk | coff of the last call
-  int32_t* order = nullptr;    // device [cand_cap / 256]
+  // the last call's table: blk [B + 1] | coff [B + 1] | pair order [P / 256]
+  int32_t* table = nullptr;    // device
+  size_t table_ints = 0;       // capacity, in int32
+  int32_t* hoff_host = nullptr;       // pinned [max_users + 1]: history offsets of the prefill
+  cudaEvent_t hoff_ready = nullptr;   // recorded behind their copy
+  int32_t* ring[kRing] = {nullptr, nullptr, nullptr, nullptr};   // pinned, table_ints each
+  cudaEvent_t ring_done[kRing] = {nullptr, nullptr, nullptr, nullptr};
+  bool ring_used[kRing] = {false, false, false, false};
+  int ring_next = 0;
   void* xblk = nullptr;        // device [cand_cap, d] io dtype: the block's residual stream
-  std::vector<int32_t> table_host;
 };
 
 namespace {
@@ -791,9 +800,15 @@ hstu_status hstu_cache_destroy(hstu_history_cache* c) {
   cudaDeviceSynchronize();
   for (void* p : c->uvqk)
     if (p != nullptr) cudaFree(p);
-  void* ptrs[] = {c->ts, c->hoff, c->table, c->order, c->xblk};
+  void* ptrs[] = {c->ts, c->hoff, c->table, c->xblk};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
+  if (c->hoff_host != nullptr) cudaFreeHost(c->hoff_host);
+  if (c->hoff_ready != nullptr) cudaEventDestroy(c->hoff_ready);
+  for (int k = 0; k < hstu_history_cache_s::kRing; ++k) {
+    if (c->ring[k] != nullptr) cudaFreeHost(c->ring[k]);
+    if (c->ring_done[k] != nullptr) cudaEventDestroy(c->ring_done[k]);
+  }
   delete c;
   return HSTU_OK;
 }
@@ -833,16 +848,22 @@ hstu_status hstu_cache_create(hstu_handle* h, int32_t num_layers, int64_t max_hi
   }
   if (e == cudaSuccess) e = hstu::alloc(&c->ts, size_t(rows_cap) * 8);
   if (e == cudaSuccess) e = cudaMemset(c->ts, 0, size_t(rows_cap) * 8);
+  c->table_ints = size_t(2 * (cfg.max_users + 1)) + size_t(cand_cap / (2 * hstu::kTile));
   if (e == cudaSuccess) e = hstu::alloc(&c->hoff, size_t(cfg.max_users + 1) * 4);
-  if (e == cudaSuccess) e = hstu::alloc(&c->table, size_t(2 * (cfg.max_users + 1)) * 4);
-  if (e == cudaSuccess) e = hstu::alloc(&c->order, size_t(cand_cap / (2 * hstu::kTile)) * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&c->table, c->table_ints * 4);
   if (e == cudaSuccess) e = hstu::alloc(&c->xblk, size_t(cand_cap) * d * io);
+  if (e == cudaSuccess)
+    e = cudaMallocHost(reinterpret_cast<void**>(&c->hoff_host), size_t(cfg.max_users + 1) * 4);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->hoff_ready, cudaEventDisableTiming);
+  for (int k = 0; e == cudaSuccess && k < hstu_history_cache_s::kRing; ++k) {
+    e = cudaMallocHost(reinterpret_cast<void**>(&c->ring[k]), c->table_ints * 4);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ring_done[k], cudaEventDisableTiming);
+  }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     hstu_cache_destroy(c);
     return HSTU_ERR_CUDA;
   }
-  c->table_host.assign(size_t(2 * (cfg.max_users + 1)), 0);
   *out = c;
   return HSTU_OK;
 }
@@ -863,6 +884,10 @@ hstu_status hstu_cache_prefill(hstu_handle* h, hstu_history_cache* c, const void
   if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(c->hoff, offsets, size_t(B + 1) * 4, cudaMemcpyDeviceToDevice, st);
+  // the history lengths on the host (pinned), for the pair order of later calls
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(c->hoff_host, offsets, size_t(B + 1) * 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaEventRecord(c->hoff_ready, st);
   if (e == cudaSuccess && T_h > 0)
     e = cudaMemcpyAsync(c->ts, ts, size_t(T_h) * 8, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
@@ -899,8 +924,12 @@ hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* 
     hstu_status s = check_weights(&layers[l]);
     if (s != HSTU_OK) return s;
   }
-  // the block layout, on the host
-  int32_t* blk = c->table_host.data();
+  // the block layout and the pair order, on the host, in a pinned slot whose
+  // previous copy has finished
+  const int slot = c->ring_next;
+  if (c->ring_used[slot] && cudaEventSynchronize(c->ring_done[slot]) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  int32_t* blk = c->ring[slot];
   int32_t* coff = blk + B + 1;
   int64_t P = 0, T_c = 0;
   for (int32_t b = 0; b < B; ++b) {
@@ -919,20 +948,38 @@ hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* 
       !hstu::aligned16(out) || !hstu::aligned16(timestamps))
     return HSTU_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaEventSynchronize(c->hoff_ready) != cudaSuccess) return HSTU_ERR_CUDA;
+  // pairs by descending history length of their user (ties by pair index):
+  // the longest-first order of the attention's work items
+  const int64_t q0 = round_pair(c->T_h);
+  const int32_t n_pairs = int32_t(P / (2 * hstu::kTile));
+  int32_t* order = coff + B + 1;
+  {
+    std::vector<std::pair<int64_t, int32_t>> key;
+    key.reserve(size_t(n_pairs));
+    for (int32_t b = 0; b < B; ++b) {
+      int64_t hl = int64_t(c->hoff_host[b + 1]) - int64_t(c->hoff_host[b]);
+      if (hl < 0) hl = 0;
+      for (int32_t k = blk[b] / (2 * hstu::kTile); k < blk[b + 1] / (2 * hstu::kTile); ++k)
+        key.emplace_back(-hl, k);
+    }
+    std::sort(key.begin(), key.end());
+    for (int32_t k = 0; k < n_pairs; ++k)
+      order[k] = int32_t(q0 / (2 * hstu::kTile)) + key[size_t(k)].second;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const hstu_config& cfg = h->cfg;
   const int64_t row_bytes = int64_t(cfg.d_model) * int64_t(hstu::elem_size(cfg.io_dtype));
-  const int64_t q0 = round_pair(c->T_h);
-  // pageable source: the copy is staged before the call returns, so the host
-  // table may be rewritten by the next call
-  cudaError_t e = cudaMemcpyAsync(c->table, c->table_host.data(), size_t(2 * (B + 1)) * 4,
-                                  cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) {
+  const size_t ints = size_t(2 * (B + 1) + n_pairs);
+  cudaError_t e = cudaMemcpyAsync(c->table, blk, ints * 4, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ring_done[slot], st);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  c->ring_used[slot] = true;
+  c->ring_next = (slot + 1) % hstu_history_cache_s::kRing;
+  {
     Timed tm(h, kBlock, st);
-    e = hstu::launch_candidate_rows(c->table, c->hoff, B, c->T_h, q0, int32_t(P), timestamps,
-                                    c->ts, h->ws.rows, c->order, st);
-    if (e == cudaSuccess)
-      e = hstu::launch_candidate_copy(c->table, B, int32_t(P), row_bytes, values, c->xblk, true, st);
+    e = hstu::launch_candidate_block(c->table, c->hoff, B, c->T_h, q0, int32_t(P), timestamps,
+                                     c->ts, h->ws.rows, row_bytes, values, c->xblk, st);
   }
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
   LayerRows R;
@@ -940,7 +987,7 @@ hstu_status hstu_cache_score(hstu_handle* h, hstu_history_cache* c, const void* 
   R.M = P;
   R.T_attn = q0 + P;
   R.num_pairs = int(P / (2 * hstu::kTile));
-  R.order = c->order;
+  R.order = c->table + 2 * (B + 1);
   R.ts = c->ts;
   for (int32_t l = 0; l < num_layers; ++l) {
     R.uvqk = c->uvqk[l];

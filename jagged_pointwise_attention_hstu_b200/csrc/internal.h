@@ -125,12 +125,14 @@ cudaError_t launch_cast_bf16(const float* x, void* xb, int64_t n, cudaStream_t s
 // serve.cu: the candidate block of a history-cache call.  table = blk[0..B]
 // (padded block starts, relative to the block, multiples of 2 * kTile) followed
 // by coff[0..B] (packed candidate offsets); hoff[0..B]: history offsets.
-constexpr int32_t kMaxCandidatePairs = 8192;   // the pair order is ranked in shared memory
-cudaError_t launch_candidate_rows(const int32_t* table, const int32_t* hoff, int32_t B,
-                                  int64_t T_h, int64_t q0, int32_t P, const int64_t* cand_ts,
-                                  int64_t* ts, RowInfo* rows, int32_t* order, cudaStream_t st);
-// to_block: packed candidate rows [T_c, row_bytes] -> block rows [P, row_bytes],
-// padding rows zeroed; else block -> packed (padding rows dropped).
+constexpr int32_t kMaxCandidatePairs = 8192;
+// Row facts and timestamps of the block rows, and the packed candidate rows
+// [T_c, row_bytes] moved into the block [P, row_bytes] (padding rows zeroed).
+cudaError_t launch_candidate_block(const int32_t* table, const int32_t* hoff, int32_t B,
+                                   int64_t T_h, int64_t q0, int32_t P, const int64_t* cand_ts,
+                                   int64_t* ts, RowInfo* rows, int64_t row_bytes, const void* src,
+                                   void* dst, cudaStream_t st);
+// Block rows back to packed order (padding dropped); to_block must be false.
 cudaError_t launch_candidate_copy(const int32_t* table, int32_t B, int32_t P, int64_t row_bytes,
                                   const void* src, void* dst, bool to_block, cudaStream_t st);
 
