@@ -113,6 +113,8 @@ def parse():
                          "16-user lognormal workload")
     ap.add_argument("--attn-bwd", action="store_true",
                     help="time the attention backward on one layer of the workload")
+    ap.add_argument("--train", action="store_true",
+                    help="forward and backward of the stack per step (layer-tokens/s)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling aid: draw only the first N layers (default: all of the "
                          "workload's layers; per-layer kernels and their sizes are unchanged)")
@@ -630,10 +632,85 @@ def run_attn_bwd(args):
     return 0
 
 
+def run_train(args):
+    """Training steps on one GPU: per step the stack's forward (keeping each
+    layer's input, U|V|Q|K and O) and its backward (every gradient), both
+    through the C ABI.  value = tokens x layers / step time."""
+    import torch
+    from jagged_pointwise_attention_hstu_b200 import hstu, runtime
+
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("--train runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.workload]
+    batch = wl.make_batch(w, num_layers=args.layers)
+    L = len(batch.layers)
+    T = batch.total_tokens
+    d = w.d_model
+    cfg = runtime.config_for(w, T, batch.num_users)
+    handle = runtime.Handle(cfg, 0)
+    db = runtime.to_device(batch, w.storage, w.compute, dev)
+    io = db.x.dtype
+    saved = {"x": [torch.empty((T, d), dtype=io, device=dev) for _ in range(L)],
+             "uvqk": [torch.empty((T, 4 * d), dtype=torch.bfloat16, device=dev) for _ in range(L)],
+             "av": [torch.empty((T, d), dtype=torch.float32, device=dev) for _ in range(L)],
+             "y": torch.empty((T, d), dtype=io, device=dev),
+             "dx": torch.empty((T, d), dtype=io, device=dev)}
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = [{"w1": torch.empty((4 * d, d), **f32), "b1": torch.empty(4 * d, **f32),
+              "w2": torch.empty((d, d), **f32), "b2": torch.empty(d, **f32),
+              "ln_gamma": torch.empty(d, **f32), "ln_beta": torch.empty(d, **f32),
+              "rab_pos": torch.empty(w.pos_buckets, **f32),
+              "rab_time": torch.empty(w.time_buckets, **f32)} for _ in range(L)]
+    dy = torch.randn((T, d), generator=torch.Generator(device=dev).manual_seed(5), device=dev,
+                     dtype=torch.float32).to(io)
+    mode = runtime.mask_mode_of(w)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(args.warmup, 0)):
+        handle.train_step(db, mode, dy, saved, grads, stream)
+    torch.cuda.synchronize(dev)
+    if handle.device_error():
+        raise RuntimeError("device error during warm-up")
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(gpu_id) as clk:
+        for s0, s1 in evs:
+            flush.fill_(1)
+            s0.record(stream)
+            handle.train_step(db, mode, dy, saved, grads, stream)
+            s1.record(stream)
+        torch.cuda.synchronize(dev)
+    if handle.device_error():
+        raise RuntimeError("device error during the timed region")
+    ms = sum(s0.elapsed_time(s1) for s0, s1 in evs) / args.steps
+    attn_fwd, gemm_fwd = workload_flops(w, batch)
+    # forward 1x; backward: attention 2.5x its forward (S recomputed, dA, dV, dK, dQ),
+    # GEMMs 2x (dG, dX, dW1, dW2) plus the recomputed f1 (0.8 of the forward GEMM flops)
+    flops = L * (3.5 * attn_fwd + 3.8 * gemm_fwd)
+    line = {
+        "metric": "HSTU training step (forward + backward) layer-tokens/s",
+        "value": T * L / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": T, "layers": L, "d_model": d,
+                   "l2": "each step timed alone after a 256 MB write"},
+        "tflops_model": flops / (ms / 1e3) / 1e12,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    handle.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.attn_bwd:
         return run_attn_bwd(args)
+    if args.train:
+        return run_train(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.serve:

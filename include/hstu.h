@@ -357,6 +357,42 @@ hstu_status hstu_attention_backward(hstu_handle* h, const void* uvqk, const void
                                     float* dk, float* dv, float* d_rab_pos, float* d_rab_time,
                                     void* stream);
 
+/* ---- Backward of one layer ----
+ * Gradients of sum(dY * Y) for Y = hstu_layer_forward(X) (equations (1)-(3)
+ * plus the residual), by the chain rule in the reverse order of the forward:
+ * f2 and the residual, the gate, the LayerNorm, the attention step
+ * (hstu_attention_backward's kernel), SiLU and f1.  Every product runs on the
+ * tensor-core GEMM (operands transposed into K-major copies where needed);
+ * H1 = X W1^T + b1 is recomputed, and the gate's statistics come from O.
+ *   values          device [T, d] io_dtype: the layer input X
+ *   uvqk, av        the forward's SiLU(X W1^T + b1) (bf16 [T, 4d]) and attention
+ *                   output O (fp32 [T, d]) for the same X (hstu_copy_intermediate
+ *                   after hstu_layer_forward)
+ *   d_out           device [T, d] io_dtype: dY
+ *   d_values        device [T, d] io_dtype: dX (may alias d_out)
+ *   grads           host pointer to device pointers, all fp32, overwritten:
+ *                   w1 [4d, d], b1 [4d], w2 [d, d], b2 [d], ln_gamma [d],
+ *                   ln_beta [d], rab_pos [pos_buckets], rab_time [time_buckets]
+ * The first call allocates the handle's backward buffers (about 68 d bytes
+ * per max_tokens row, plus the transposed weights); compute dtype BF16 only. */
+typedef struct {
+  float* w1;
+  float* b1;
+  float* w2;
+  float* b2;
+  float* ln_gamma;
+  float* ln_beta;
+  float* rab_pos;
+  float* rab_time;
+} hstu_layer_grads;
+
+hstu_status hstu_layer_backward(hstu_handle* h, const void* values, const void* uvqk,
+                                const float* av, const void* d_out, int64_t total_tokens,
+                                const int32_t* seq_offsets, int32_t num_users,
+                                const int64_t* timestamps, const hstu_layer_weights* weights,
+                                hstu_mask_mode mask_mode, const int32_t* num_candidates,
+                                void* d_values, const hstu_layer_grads* grads, void* stream);
+
 /* ---- Inspection entry points for tests (same library, same kernels) ---- */
 
 typedef enum {

@@ -244,6 +244,11 @@ hstu_status hstu_destroy(hstu_handle* h) {
                   ws.counters, ws.error, ws.thresholds, ws.time_lut, ws.thr32};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
+  hstu::BwdWorkspace& bw = h->bwd;
+  void* bptrs[] = {bw.xb, bw.dyb, bw.w1t, bw.w2t, bw.dg, bw.du, bw.dO, bw.g, bw.dq, bw.dk,
+                   bw.dv, bw.h1, bw.dh1, bw.dh1t, bw.xt, bw.dyt, bw.gt, bw.zeros};
+  for (void* p : bptrs)
+    if (p != nullptr) cudaFree(p);
   if (h->timer.created)
     for (int i = 0; i < 2 * hstu::KernelTimer::kMax; ++i) cudaEventDestroy(h->timer.ev[i]);
   delete h;
@@ -1120,5 +1125,184 @@ extern "C" hstu_status hstu_attention_backward(
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
   e = hstu::launch_attention_bwd_tc(a, st);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Backward of one layer
+namespace {
+
+cudaError_t bwd_alloc(hstu_handle* h) {
+  hstu::BwdWorkspace& b = h->bwd;
+  if (b.ready) return cudaSuccess;
+  const size_t T = size_t(h->cfg.max_tokens), d = size_t(h->cfg.d_model);
+  const size_t T64 = (T + 63) / 64 * 64;
+  cudaError_t e = cudaSuccess;
+  auto get = [&](void** p, size_t bytes) {
+    if (e == cudaSuccess) e = hstu::alloc(p, bytes > 0 ? bytes : 16);
+  };
+  get(&b.xb, T * d * 2);
+  get(&b.dyb, T * d * 2);
+  get(&b.w1t, 4 * d * d * 2);
+  get(&b.w2t, d * d * 2);
+  get(reinterpret_cast<void**>(&b.dg), T * d * 4);
+  get(reinterpret_cast<void**>(&b.du), T * d * 4);
+  get(&b.dO, T * d * 2);
+  get(&b.g, T * d * 2);
+  get(reinterpret_cast<void**>(&b.dq), T * d * 4);
+  get(reinterpret_cast<void**>(&b.dk), T * d * 4);
+  get(reinterpret_cast<void**>(&b.dv), T * d * 4);
+  get(reinterpret_cast<void**>(&b.h1), T * 4 * d * 4);
+  get(&b.dh1, T * 4 * d * 2);
+  get(&b.dh1t, 4 * d * T64 * 2);
+  get(&b.xt, d * T64 * 2);
+  get(&b.dyt, d * T64 * 2);
+  get(&b.gt, d * T64 * 2);
+  get(reinterpret_cast<void**>(&b.zeros), 4 * d * 4);
+  if (e == cudaSuccess) e = cudaMemset(b.zeros, 0, 4 * d * 4);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) b.ready = true;
+  return e;
+}
+
+// out (fp32 [M, N], zeroed first) = A [M, K] B[N, K]^T (+ bias), both K-major bf16
+cudaError_t gemm_f32(hstu_handle* h, const void* a, const void* b, int64_t M, int N, int K,
+                     const float* bias, float* out, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(out, 0, size_t(M) * size_t(N) * 4, st);
+  if (e != cudaSuccess) return e;
+  hstu::GemmArgs g;
+  g.a = a;
+  g.b = b;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.epi = hstu::Epi::kBiasResidual;
+  g.bias = bias;
+  g.out = out;
+  g.residual = out;   // zero: out = A B^T + bias
+  g.io_fp32 = 1;
+  g.out_bf16 = nullptr;
+  return hstu::launch_gemm_tc(g, h->num_sms, st, h->ws.error);
+}
+
+}  // namespace
+
+extern "C" hstu_status hstu_layer_backward(
+    hstu_handle* h, const void* values, const void* uvqk, const float* av, const void* d_out,
+    int64_t T, const int32_t* offsets, int32_t B, const int64_t* ts,
+    const hstu_layer_weights* w, hstu_mask_mode mode, const int32_t* ncand, void* d_values,
+    const hstu_layer_grads* gr, void* stream) {
+  hstu_status s = check_common(h, values, T, offsets, B, ts, mode, ncand, d_values);
+  if (s != HSTU_OK) return s;
+  s = check_weights(w);
+  if (s != HSTU_OK) return s;
+  if (h->cfg.compute_dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (gr == nullptr) return HSTU_ERR_INVALID_ARG;
+  const void* gp[] = {gr->w1, gr->b1, gr->w2, gr->b2, gr->ln_gamma, gr->ln_beta, gr->rab_pos,
+                      gr->rab_time};
+  for (const void* q : gp)
+    if (q == nullptr || !hstu::aligned16(q)) return HSTU_ERR_INVALID_ARG;
+  if (T > 0) {
+    const void* ip[] = {uvqk, av, d_out};
+    for (const void* q : ip)
+      if (q == nullptr || !hstu::aligned16(q)) return HSTU_ERR_INVALID_ARG;
+  }
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (bwd_alloc(h) != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu_config& c = h->cfg;
+  const int d = c.d_model;
+  const bool io32 = c.io_dtype == HSTU_DTYPE_FP32;
+  hstu::BwdWorkspace& b = h->bwd;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t T64 = (T + 63) / 64 * 64;
+  cudaError_t e = cudaSuccess;
+  // gradients that are sums start at zero
+  e = cudaMemsetAsync(gr->b1, 0, size_t(4 * d) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->b2, 0, size_t(d) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->ln_gamma, 0, size_t(d) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->ln_beta, 0, size_t(d) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->rab_pos, 0, size_t(c.pos_buckets) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->rab_time, 0, size_t(c.time_buckets) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->w1, 0, size_t(4 * d) * size_t(d) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->w2, 0, size_t(d) * size_t(d) * 4, st);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (T == 0) return HSTU_OK;
+  // bf16 operands
+  const void* xb = values;
+  const void* dyb = d_out;
+  if (io32) {
+    e = hstu::launch_cast_bf16(static_cast<const float*>(values), b.xb, T * d, st);
+    if (e == cudaSuccess) e = hstu::launch_cast_bf16(static_cast<const float*>(d_out), b.dyb, T * d, st);
+    xb = b.xb;
+    dyb = b.dyb;
+  }
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(w->w2, false, d, d, d, b.w2t, d, st);
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(w->w1, false, 4 * d, d, d, b.w1t, 4 * d, st);
+  // dG = dY W2; everything else that reads dY happens before dX is written,
+  // since d_values may alias d_out
+  if (e == cudaSuccess) e = gemm_f32(h, dyb, b.w2t, T, d, d, b.zeros, b.dg, st);
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(dyb, false, T, d, d, b.dyt, T64, st);
+  if (e == cudaSuccess) e = hstu::launch_colsum(d_out, io32, T, d, gr->b2, h->num_sms, st);
+  // the gate and the LayerNorm
+  if (e == cudaSuccess)
+    e = hstu::launch_ln_gate_bwd(b.dg, uvqk, av, w->ln_gamma, w->ln_beta, T, d, c.ln_eps, b.du,
+                                 b.dO, b.g, gr->ln_gamma, gr->ln_beta, h->num_sms, st);
+  // the attention step (its schedule, then the backward kernel)
+  if (e == cudaSuccess) e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(b.dq, 0, size_t(T) * d * 4, st);
+  if (e == cudaSuccess) {
+    hstu::AttnBwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.uvqk = uvqk;
+    a.dO = b.dO;
+    a.rows = h->ws.rows;
+    a.offsets = offsets;
+    a.B = B;
+    a.ts = ts;
+    a.thresholds = h->ws.thresholds;
+    a.rab_pos = w->rab_pos;
+    a.rab_time = w->rab_time;
+    a.counters = h->ws.counters;
+    a.error = h->ws.error;
+    a.dq = b.dq;
+    a.dk = b.dk;
+    a.dv = b.dv;
+    a.d_rab_pos = gr->rab_pos;
+    a.d_rab_time = gr->rab_time;
+    a.T = T;
+    a.d = d;
+    a.H = c.num_heads;
+    a.hd = c.head_dim;
+    a.pos_clamp = c.pos_clamp;
+    a.time_buckets = c.time_buckets;
+    a.n_norm_fixed = c.n_norm;
+    e = hstu::launch_attention_bwd_tc(a, st);
+  }
+  // SiLU: H1 recomputed, dH1 = dZ (.) SiLU'(H1), b1 gradient
+  if (e == cudaSuccess) e = gemm_f32(h, xb, w->w1, T, 4 * d, d, w->b1, b.h1, st);
+  if (e == cudaSuccess)
+    e = hstu::launch_silu_bwd(b.du, b.dv, b.dq, b.dk, b.h1, T, d, b.dh1, gr->b1, h->num_sms, st);
+  // dX = dH1 W1 + dY
+  if (e == cudaSuccess) {
+    hstu::GemmArgs g;
+    g.a = b.dh1;
+    g.b = b.w1t;
+    g.M = T;
+    g.N = d;
+    g.K = 4 * d;
+    g.epi = hstu::Epi::kBiasResidual;
+    g.bias = b.zeros;
+    g.out = d_values;
+    g.residual = d_out;
+    g.io_fp32 = io32 ? 1 : 0;
+    g.out_bf16 = nullptr;
+    e = hstu::launch_gemm_tc(g, h->num_sms, st, h->ws.error);
+  }
+  // weight gradients over the tokens: dW1 = dH1^T X, dW2 = dY^T G, b2
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(b.dh1, false, T, 4 * d, 4 * d, b.dh1t, T64, st);
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(xb, false, T, d, d, b.xt, T64, st);
+  if (e == cudaSuccess) e = hstu::launch_transpose_bf16(b.g, false, T, d, d, b.gt, T64, st);
+  if (e == cudaSuccess) e = gemm_f32(h, b.dh1t, b.xt, 4 * d, d, int(T64), b.zeros, gr->w1, st);
+  if (e == cudaSuccess) e = gemm_f32(h, b.dyt, b.gt, d, d, int(T64), b.zeros, gr->w2, st);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }

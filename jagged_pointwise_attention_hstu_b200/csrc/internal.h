@@ -98,8 +98,35 @@ struct KernelTimer {
 };
 }  // namespace hstu
 
+namespace hstu {
+// Buffers of the layer backward, allocated on its first call (sized by the
+// handle's max_tokens).
+struct BwdWorkspace {
+  void* xb = nullptr;       // [T, d] bf16: X for the products
+  void* dyb = nullptr;      // [T, d] bf16: dY for the products
+  void* w1t = nullptr;      // [d, 4d] bf16: W1^T
+  void* w2t = nullptr;      // [d, d] bf16: W2^T
+  float* dg = nullptr;      // [T, d]
+  float* du = nullptr;      // [T, d]
+  void* dO = nullptr;       // [T, d] bf16
+  void* g = nullptr;        // [T, d] bf16: N (.) U
+  float* dq = nullptr;      // [T, d]
+  float* dk = nullptr;      // [T, d]
+  float* dv = nullptr;      // [T, d]
+  float* h1 = nullptr;      // [T, 4d]: X W1^T + b1
+  void* dh1 = nullptr;      // [T, 4d] bf16
+  void* dh1t = nullptr;     // [4d, T64] bf16
+  void* xt = nullptr;       // [d, T64] bf16
+  void* dyt = nullptr;      // [d, T64] bf16
+  void* gt = nullptr;       // [d, T64] bf16
+  float* zeros = nullptr;   // [4d]
+  bool ready = false;
+};
+}  // namespace hstu
+
 struct hstu_handle_s {
   hstu_config cfg;
+  hstu::BwdWorkspace bwd;
   hstu::KernelTimer timer;
   int device = 0;
   int num_sms = 148;
@@ -229,6 +256,19 @@ struct AttnBwdArgs {
   int pos_clamp, time_buckets, n_norm_fixed;
 };
 cudaError_t launch_attention_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
+
+// bwd_aux.cu: memory-bound steps of the layer backward
+cudaError_t launch_ln_gate_bwd(const float* dG, const void* uvqk, const float* av,
+                               const float* gamma, const float* beta, int64_t T, int d, float eps,
+                               float* dU, void* dO, void* G, float* dgamma, float* dbeta,
+                               int num_sms, cudaStream_t st);
+cudaError_t launch_silu_bwd(const float* dU, const float* dV, const float* dQ, const float* dK,
+                            const float* H1, int64_t T, int d, void* dH1, float* db1, int num_sms,
+                            cudaStream_t st);
+cudaError_t launch_colsum(const void* src, bool fp32, int64_t T, int n, float* out, int num_sms,
+                          cudaStream_t st);
+cudaError_t launch_transpose_bf16(const void* src, bool fp32, int64_t R, int C, int64_t lds,
+                                  void* dst, int64_t ldd, cudaStream_t st);
 
 // ln_gate.cu
 cudaError_t launch_ln_gate(const float* av, const void* uvqk, void* g, const float* gamma,

@@ -47,6 +47,12 @@ class HstuError(RuntimeError):
         self.status = status
 
 
+class hstu_layer_grads(ctypes.Structure):
+    _fields_ = [("w1", c_void_p), ("b1", c_void_p), ("w2", c_void_p), ("b2", c_void_p),
+                ("ln_gamma", c_void_p), ("ln_beta", c_void_p), ("rab_pos", c_void_p),
+                ("rab_time", c_void_p)]
+
+
 class hstu_config(ctypes.Structure):
     _fields_ = [("d_model", c_int32), ("num_heads", c_int32), ("head_dim", c_int32),
                 ("io_dtype", c_int), ("compute_dtype", c_int), ("n_norm", c_int32),
@@ -110,6 +116,10 @@ def load() -> ctypes.CDLL:
                                             c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_void_p]),
+        "hstu_layer_backward": (c_int, [H, c_void_p, c_void_p, c_void_p, c_void_p, c_int64,
+                                        c_void_p, c_int32, c_void_p,
+                                        POINTER(hstu_layer_weights), c_int, c_void_p, c_void_p,
+                                        POINTER(hstu_layer_grads), c_void_p]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -298,6 +308,20 @@ def hstu_attention_backward(handle, uvqk, d_out, total_tokens: int, seq_offsets,
                                           _ptr(rab_time), _ptr(dq), _ptr(dk), _ptr(dv),
                                           _ptr(d_rab_pos), _ptr(d_rab_time), _stream_ptr(stream)),
            "hstu_attention_backward")
+
+
+def hstu_layer_backward(handle, values, uvqk, av, d_out, total_tokens: int, seq_offsets,
+                        num_users: int, timestamps, weights: hstu_layer_weights, mask_mode: int,
+                        num_candidates, d_values, grads: dict, stream=None) -> None:
+    """grads: dict of fp32 device tensors w1, b1, w2, b2, ln_gamma, ln_beta, rab_pos, rab_time."""
+    g = hstu_layer_grads(*[_ptr(grads[k]) for k in ("w1", "b1", "w2", "b2", "ln_gamma",
+                                                    "ln_beta", "rab_pos", "rab_time")])
+    _check(load().hstu_layer_backward(handle, _ptr(values), _ptr(uvqk), _ptr(av), _ptr(d_out),
+                                      total_tokens, _ptr(seq_offsets), num_users,
+                                      _ptr(timestamps), ctypes.byref(weights), mask_mode,
+                                      _ptr(num_candidates), _ptr(d_values), ctypes.byref(g),
+                                      _stream_ptr(stream)),
+           "hstu_layer_backward")
 
 
 KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2", "block")

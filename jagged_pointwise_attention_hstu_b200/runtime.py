@@ -123,6 +123,41 @@ class Handle:
                                     stream)
         return out
 
+    def train_step(self, db: DeviceBatch, mask_mode: int, dy: torch.Tensor, saved: dict,
+                   grads: List[dict], stream=None) -> torch.Tensor:
+        """One forward and backward pass of the stack through the C ABI.
+
+        The forward runs layer by layer and keeps each layer's input and the
+        U|V|Q|K and O the backward reads (``saved``: preallocated lists "x",
+        "uvqk", "av" of per-layer device tensors, "y" and "dx" [T, d]); the
+        backward walks the
+        layers in reverse with hstu_layer_backward, filling ``grads[l]`` and
+        returning dX of the stack's input."""
+        if stream is None:
+            stream = torch.cuda.current_stream(dy.device)
+        T = db.total_tokens
+        L = len(db.layers)
+        saved["x"][0].copy_(db.x)
+        for l in range(L):
+            out = saved["x"][l + 1] if l + 1 < L else saved["y"]
+            hstu.hstu_layer_forward(self.h, saved["x"][l], T, db.seq_offsets, db.num_users,
+                                    db.timestamps, db.layers[l].struct(), mask_mode,
+                                    db.num_candidates, out, stream)
+            u, a = saved["uvqk"][l], saved["av"][l]
+            hstu.hstu_copy_intermediate(self.h, hstu.HSTU_TENSOR_UVQK, u,
+                                        u.numel() * u.element_size(), stream)
+            hstu.hstu_copy_intermediate(self.h, hstu.HSTU_TENSOR_AV, a,
+                                        a.numel() * a.element_size(), stream)
+        g = dy
+        for l in reversed(range(L)):
+            dx = saved["dx"]
+            hstu.hstu_layer_backward(self.h, saved["x"][l], saved["uvqk"][l], saved["av"][l], g,
+                                     T, db.seq_offsets, db.num_users, db.timestamps,
+                                     db.layers[l].struct(), mask_mode, db.num_candidates, dx,
+                                     grads[l], stream)
+            g = dx
+        return g
+
     def intermediate(self, which: int, T: int) -> torch.Tensor:
         d = self.cfg.d_model
         cdt = torch.bfloat16 if self.cfg.compute_dtype == hstu.HSTU_DTYPE_BF16 else torch.float32
