@@ -288,7 +288,8 @@ def run_reference(args):
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "sample": f"1 layer over user 0's first {prefix} tokens per step"},
@@ -705,8 +706,54 @@ def run_train(args):
     return 0
 
 
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n, script, argv, timeout_s=1800):
+    """Runs `script argv` as n ranks of one node (torch.distributed.run, one
+    process per GPU, rendezvous on 127.0.0.1) and returns the launcher's exit
+    status (non-zero when any rank fails or the timeout ends the job)."""
+    cmd = ["timeout", "-k", "60", str(int(timeout_s)), sys.executable, "-m",
+           "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={int(n)}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), script] + list(argv)
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT")}
+    return subprocess.run(cmd, env=env).returncode
+
+
+def launch_check(args):
+    """--gpus N without a launcher: start N ranks here.  Returns an exit status
+    to end with, or None when this process is the rank that should run."""
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is not None:
+        if int(world_env) != args.gpus:
+            print(f"--gpus {args.gpus} but WORLD_SIZE={world_env}", file=sys.stderr)
+            return 2
+        return None
+    if args.gpus <= 1:
+        return None
+    if args.serve or args.sl or args.attn_bwd or args.train:
+        print("--serve, --sl, --attn-bwd and --train run on one GPU", file=sys.stderr)
+        return 2
+    if args.impl == "ours":
+        import torch
+        have = torch.cuda.device_count() if torch.cuda.is_available() else 0
+        if have < args.gpus:
+            print(f"--gpus {args.gpus}: only {have} CUDA device(s) visible; not running on fewer",
+                  file=sys.stderr)
+            return 2
+    return spawn_ranks(args.gpus, os.path.abspath(__file__), sys.argv[1:])
+
+
 def main():
     args = parse()
+    rc = launch_check(args)
+    if rc is not None:
+        return rc
     if args.attn_bwd:
         return run_attn_bwd(args)
     if args.train:

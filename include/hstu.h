@@ -181,14 +181,16 @@ hstu_status hstu_get_kernel_timing(hstu_handle* h, double* total_ms, int64_t* la
 
 /* ---- Attention without allocation ----
  * The pages have no counterpart of this entry point: it is an interface of
- * this library for callers that may not allocate at call time.  It runs the
- * attention step of equation (2) alone -- the scheduler and the fused
- * tensor-core attention kernel of the BF16 path, the same kernels that
- * hstu_layer_forward launches -- with every piece of scratch (per-token row
- * facts, pair order and cost, counters, the error word, the time-bucket
- * tables) in one fixed file-scope device array of this library, about 1 MiB
- * per device, instead of a handle's workspace.  Neither the call nor anything
- * it calls allocates host or device memory.
+ * this library for callers that may not allocate device memory at call time
+ * -- for instance code running inside a region where cudaMalloc is not
+ * allowed, or a host framework that owns every allocation.  It runs the
+ * attention step alone -- the scheduler and the fused tensor-core attention
+ * kernel of the BF16 path, the same kernels that hstu_layer_forward launches --
+ * with every piece of scratch (per-token row facts, pair order and cost,
+ * counters, the error word, the time-bucket tables) in one fixed file-scope
+ * device array of this library, about 1 MiB per device, instead of a handle's
+ * workspace.  Apart from the set-up below, neither the call nor anything it
+ * calls allocates host or device memory.
  *   cfg            host; uses d_model, num_heads, head_dim, n_norm, pos_buckets,
  *                  pos_clamp, time_buckets and time_log_div; compute_dtype must be
  *                  BF16 and head_dim 64 or 128 (else HSTU_ERR_UNSUPPORTED);
@@ -201,14 +203,22 @@ hstu_status hstu_get_kernel_timing(hstu_handle* h, double* total_ms, int64_t* la
  *                  as for hstu_layer_forward
  *   rab_pos        device fp32 [pos_buckets]
  *   rab_time       device fp32 [time_buckets]
- *   av             device fp32 [T, d]: O of equation (2), divided by n_norm
+ *   av             device fp32 [T, d]: for every row i and head, the sum over the
+ *                  visible keys j of SiLU(q_i.k_j + rab_pos[p(i,j)] + rab_time[t(i,j)]) v_j,
+ *                  divided by n_norm once -- the tensor HSTU_TENSOR_AV of a layer
+ *                  forward on the same U|V|Q|K
  *   device_error   device int32 or NULL: overwritten with this call's
  *                  HSTU_DEVERR_* bits (0 = none), in stream order
  *   stream         cudaStream_t or NULL
  * Set-up: the first call on a device looks up the address of the scratch
  * array there (cudaGetSymbolAddress, checked; HSTU_ERR_CUDA on failure) and
- * caches it; make that first call outside any stream capture.  The bucket
- * tables are rebuilt on the host when time_log_div or time_buckets changes.
+ * caches it.  With CUDA's lazy module loading that first call may also load
+ * this library's device code, array included, which allocates: it is the only
+ * call that can.  Make one warm-up call per device before any region where
+ * allocation or stream capture is not allowed.  A device reset
+ * (cudaDeviceReset) invalidates the cached address: do not call this entry
+ * point on that device again in the same process.  The bucket tables are
+ * rebuilt on the host when time_log_div or time_buckets changes.
  * Every call first clears the scratch that must start at zero (the counters
  * and the error word) and rewrites the tables, in stream order.
  * The scratch is one per device and process: two calls on one device whose
@@ -335,6 +345,27 @@ hstu_status hstu_stochastic_length(const int32_t* seq_offsets, int32_t num_users
                                    int64_t* out_index, void* out_values,
                                    int64_t* out_timestamps, void* scratch,
                                    int32_t* device_error, void* stream);
+
+/* ---- The attention step alone ----
+ * Equation (2) of the layer (blog "Generative Recommendation 16: HSTU",
+ * section "HSTU Layer 到底改了什么"; no softmax, section "不对序列做 softmax")
+ * on U|V|Q|K the caller supplies: for every row i,
+ *   av[i, h-th head] = sum over visible j of SiLU(q_i.k_j + rab_pos[p(i,j)] + rab_time[t(i,j)]) v_j / n_norm
+ * with the same jagged schedule, masks, buckets and kernels as hstu_layer_forward
+ * (BF16 compute: the tensor-core kernel; FP32 compute: the fp32 kernel).
+ *   uvqk            device [T, 4d] compute dtype: columns U | V | Q | K (V, Q, K read)
+ *   rab_pos         device fp32 [pos_buckets]
+ *   rab_time        device fp32 [time_buckets]
+ *   av              device fp32 [T, d] (overwritten; the tensor HSTU_TENSOR_AV of a
+ *                   layer forward on the same U|V|Q|K)
+ * Other arguments as for hstu_layer_forward; uses the handle's workspace (its
+ * row facts and work order), so calls on one handle must not overlap.
+ * Asynchronous on `stream`; device-side input errors go to the handle's error word. */
+hstu_status hstu_attention_forward(hstu_handle* h, const void* uvqk, int64_t total_tokens,
+                                   const int32_t* seq_offsets, int32_t num_users,
+                                   const int64_t* timestamps, hstu_mask_mode mask_mode,
+                                   const int32_t* num_candidates, const float* rab_pos,
+                                   const float* rab_time, float* av, void* stream);
 
 /* ---- Backward of the attention step ----
  * Gradients of sum(dO * O) for O of equation (2), computed by the handle's

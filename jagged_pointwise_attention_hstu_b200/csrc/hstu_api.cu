@@ -1077,6 +1077,59 @@ hstu_status hstu_stochastic_length(const int32_t* offsets, int32_t B, int64_t T,
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
+// The attention step alone, on the handle's workspace
+extern "C" hstu_status hstu_attention_forward(hstu_handle* h, const void* uvqk, int64_t T,
+                                              const int32_t* offsets, int32_t B,
+                                              const int64_t* ts, hstu_mask_mode mode,
+                                              const int32_t* ncand, const float* rab_pos,
+                                              const float* rab_time, float* av, void* stream) {
+  hstu_status s = check_common(h, uvqk, T, offsets, B, ts, mode, ncand, av);
+  if (s != HSTU_OK) return s;
+  if (T > 0 && (rab_pos == nullptr || rab_time == nullptr || !hstu::aligned16(rab_pos) ||
+                !hstu::aligned16(rab_time)))
+    return HSTU_ERR_INVALID_ARG;
+  if (T == 0) return HSTU_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  {
+    Timed tm(h, kSchedule, st);
+    e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
+  }
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu_config& c = h->cfg;
+  hstu::AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.uvqk = uvqk;
+  a.av = av;
+  a.rows = h->ws.rows;
+  a.order = h->ws.qtile_order;
+  a.ts = ts;
+  a.thresholds = h->ws.thresholds;
+  a.time_lut = h->ws.time_lut;
+  a.thr32 = h->ws.thr32;
+  a.lut_exact = c.time_log_div > 0.2232 ? 1 : 0;
+  a.rab_pos = rab_pos;
+  a.rab_time = rab_time;
+  a.counters = h->ws.counters;
+  a.error = h->ws.error;
+  a.T = T;
+  a.d = c.d_model;
+  a.H = c.num_heads;
+  a.hd = c.head_dim;
+  a.pos_clamp = c.pos_clamp;
+  a.time_buckets = c.time_buckets;
+  a.n_norm_fixed = c.n_norm;
+  a.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
+  {
+    Timed tm(h, kAttention, st);
+    e = c.compute_dtype == HSTU_DTYPE_FP32 ? hstu::launch_attention_f32(a, st)
+                                           : hstu::launch_attention_tc(a, st, false);
+  }
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
 // Backward of the attention step
 extern "C" hstu_status hstu_attention_backward(
     hstu_handle* h, const void* uvqk, const void* d_out, int64_t T, const int32_t* offsets,

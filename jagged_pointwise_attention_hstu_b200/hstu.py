@@ -112,6 +112,9 @@ def load() -> ctypes.CDLL:
                                            c_int32, c_double, c_void_p, c_int64, c_void_p,
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                            c_void_p, c_void_p]),
+        "hstu_attention_forward": (c_int, [H, c_void_p, c_int64, c_void_p, c_int32, c_void_p,
+                                           c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p]),
         "hstu_attention_backward": (c_int, [H, c_void_p, c_void_p, c_int64, c_void_p, c_int32,
                                             c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -297,6 +300,16 @@ def hstu_stochastic_length(seq_offsets, num_users: int, total_tokens: int, user_
                                          _ptr(out_timestamps), _ptr(scratch),
                                          _ptr(device_error), _stream_ptr(stream)),
            "hstu_stochastic_length")
+
+
+def hstu_attention_forward(handle, uvqk, total_tokens: int, seq_offsets, num_users: int,
+                           timestamps, mask_mode: int, num_candidates, rab_pos, rab_time, av,
+                           stream=None) -> None:
+    _check(load().hstu_attention_forward(handle, _ptr(uvqk), total_tokens, _ptr(seq_offsets),
+                                         num_users, _ptr(timestamps), mask_mode,
+                                         _ptr(num_candidates), _ptr(rab_pos), _ptr(rab_time),
+                                         _ptr(av), _stream_ptr(stream)),
+           "hstu_attention_forward")
 
 
 def hstu_attention_backward(handle, uvqk, d_out, total_tokens: int, seq_offsets, num_users: int,

@@ -74,17 +74,18 @@ def _rms(x):
     return float(np.sqrt(np.mean(np.asarray(x, np.float64) ** 2))) if np.size(x) else 0.0
 
 
-@pytest.mark.parametrize("mask,lengths,ncand,H", [
-    ("causal", [1, 127, 128, 129, 300, 0, 5], None, 2),
-    ("causal", [255, 256, 257], None, 4),
-    ("mfalcon", [300, 140, 260], [100, 140, 129], 4),
+@pytest.mark.parametrize("mask,lengths,ncand,H,n_norm", [
+    ("causal", [1, 127, 128, 129, 300, 0, 5], None, 2, 512),
+    ("causal", [255, 256, 257], None, 4, 512),
+    ("mfalcon", [300, 140, 260], [100, 140, 129], 4, 512),
+    # n_norm = the longest user of the batch, found on the device by the schedule
+    ("causal", [40, 300, 0, 129], None, 2, 0),
 ])
-def test_attention_backward_teacher_forced(mask, lengths, ncand, H):
+def test_attention_backward_teacher_forced(mask, lengths, ncand, H, n_norm):
     d = 256
     batch = wl.make_custom_batch(lengths, d, H, seed=sum(lengths) + H, num_candidates=ncand,
                                  weight_scale=0.05, rab_scale=1.0, random_affine=True,
                                  timestamp_gap=900.0)
-    n_norm = 512
     cfg_gpu = hstu.make_config(d, H, io_dtype=hstu.HSTU_DTYPE_BF16,
                                compute_dtype=hstu.HSTU_DTYPE_BF16, n_norm=n_norm, pos_buckets=129,
                                pos_clamp=128, time_buckets=128, time_log_div=0.301, ln_eps=1e-5,

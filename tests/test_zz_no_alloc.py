@@ -1,10 +1,11 @@
 """The no-allocation attention entry point against the handle path.
 
-hstu_attention_noalloc runs the scheduler and the fused attention kernel with
-their scratch in a fixed device array of the library.  Given the U, V, Q, K
-that hstu_layer_forward produced, it must give that call's attention output
-(equation (2) of the HSTU layer) bit for bit, call after call, while the
-configuration and the batch change between calls."""
+hstu_attention_noalloc is for callers that may not allocate device memory
+while they run (the scratch lives in a fixed device array of the library).
+Given the U, V, Q, K that hstu_layer_forward produced, it must give that
+call's attention output bit for bit, call after call, while the configuration
+and the batch change between calls -- up to the capacity limit of the array
+-- and a warm call must leave the device's free memory unchanged."""
 import pytest
 import torch
 
@@ -17,6 +18,8 @@ pytestmark = pytest.mark.gpu
 CASES = [
     ([300, 1, 0, 517, 129, 64], None, 256, 2, 0.301, 128, 0, 128),
     ([400, 77, 250], [50, 0, 10], 256, 4, 0.2, 64, 700, 64),
+    # the capacity limit: HSTU_NOALLOC_MAX_TOKENS tokens, the row facts fill their slot
+    ([8192] * 8, None, 256, 2, 0.301, 128, 8192, 1024),
 ]
 
 
@@ -93,3 +96,38 @@ def test_noalloc_error_word_starts_at_zero_on_every_call():
     av, err = _noalloc(cfg, db, uvqk, mode)
     assert err == 0
     assert torch.equal(av, av_ref)
+
+
+def test_noalloc_at_the_capacity_limit_and_allocation_free_when_warm():
+    batch, cfg, mode = _case(2, 13)
+    assert batch.total_tokens == hstu.HSTU_NOALLOC_MAX_TOKENS
+    db, uvqk, av_ref = _handle_path(batch, cfg, mode)
+    av, err = _noalloc(cfg, db, uvqk, mode)      # warm call
+    assert err == 0
+    assert torch.equal(av, av_ref)
+    out = torch.full_like(av, float("nan"))
+    dev_err = torch.full((1,), -1, dtype=torch.int32, device="cuda:0")
+    lp = db.layers[0]
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    hstu.hstu_attention_noalloc(cfg, uvqk, batch.total_tokens, db.seq_offsets, db.num_users,
+                                db.timestamps, mode, db.num_candidates, lp.rab_pos, lp.rab_time,
+                                out, dev_err, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert int(dev_err.item()) == 0
+    assert torch.equal(out, av_ref)
+
+
+def test_noalloc_of_an_empty_batch():
+    batch, cfg, mode = _case(0, 11)
+    offs = torch.zeros(1, dtype=torch.int32, device="cuda:0")
+    err = torch.full((1,), -1, dtype=torch.int32, device="cuda:0")
+    hstu.hstu_attention_noalloc(cfg, None, 0, offs, 0, None, hstu.HSTU_MASK_CAUSAL, None, None,
+                                None, None, err, torch.cuda.current_stream())
+    offs3 = torch.zeros(4, dtype=torch.int32, device="cuda:0")
+    hstu.hstu_attention_noalloc(cfg, None, 0, offs3, 3, None, hstu.HSTU_MASK_CAUSAL, None, None,
+                                None, None, err, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
