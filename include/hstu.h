@@ -162,6 +162,19 @@ hstu_status hstu_get_device_error(hstu_handle* h, int32_t* bits);
  * gap below 2^62 reaches k; out[0] = 0.  bucket(dt) = #{k >= 1 : dt >= out[k]}. */
 hstu_status hstu_time_bucket_thresholds(double time_log_div, int32_t num_buckets, int64_t* out);
 
+/* ---- Bounded waits ----
+ * Every pipeline wait of the tensor-core kernels (a TMA load landing, an MMA
+ * finishing, a row group handing over its scores) gives up after a bound of
+ * SM cycles; the kernel then sets HSTU_DEVERR_TIMEOUT in the handle's error
+ * word, still waits (with the default bound) for the copies and MMAs it has
+ * issued, frees its tensor memory and returns, so the context stays usable
+ * and out is undefined.  This sets the bound for the handle's later launches
+ * of the f1 / f2 GEMMs and the attention kernel; 0 restores the default of
+ * 2^31 cycles (about a second).  A bound of a few cycles makes every launch
+ * give up: the failure path can be exercised without a fault.
+ * HSTU_ERR_INVALID_ARG for a NULL handle or a negative bound. */
+hstu_status hstu_set_wait_limit(hstu_handle* h, int64_t cycles);
+
 /* ---- Kernel timing (CUDA events on the launching stream) ----
  * When enabled, every kernel the handle launches is bracketed by a pair of
  * CUDA events recorded on the call's stream; the pairs are read back by

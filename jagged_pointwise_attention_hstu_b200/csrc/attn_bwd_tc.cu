@@ -5,31 +5,42 @@
 // a = vis * SiLU(s) / n_norm, O = a V, the gradients of sum(dO * O) are
 //     dV = a^T dO,  dA = dO V^T,  dS = vis * dA * SiLU'(s) / n_norm,
 //     dQ = dS K,    dK = dS^T Q,
-// and every entry of rab_pos / rab_time collects dS of each visible
-// (query, key, head) that reads it.  SiLU acts on each score alone (same blog,
-// section "不对序列做 softmax"), so there are no row statistics to keep from
-// the forward: S is recomputed tile by tile.
+// with SiLU'(s) = sig(s) (1 + s (1 - sig(s))), and every entry of rab_pos /
+// rab_time collects dS of each visible (query, key, head) that reads it.  SiLU
+// acts on each score alone (same blog, section "不对序列做 softmax"): there are
+// no row statistics to keep from the forward, so S is recomputed tile by tile.
 //
-// One CTA per (128-key tile, head), 256 threads:
-//   warp 0      TMA: the key tile's K, V and key timestamps once, then per
-//               query tile its Q and dO (single buffers)
-//   warp 1      tensor-memory allocation and MMA issue:
-//                 S  = Q K^T, dA = dO V^T          (SS, both K-major)
-//                 dV += P^T dO, dK += dS^T Q       (A = P or dS read M-major
-//                                                   from shared memory, B N-major)
-//                 dQ = dS K                        (A = dS K-major, B = K N-major)
-//   warps 4-7   one query row per thread: P = a and dS from S and dA, written
-//               as bf16 into 128-byte-swizzled shared tiles; the bias
-//               gradients into shared accumulators; dQ added to global fp32
-//               (reductions); at the end one key row per thread: dK and dV
-//               of the key tile stored as fp32.
-// Query tiles visited by key tile kt: [kt, end of the user owning the tile's
-// last row) -- a query sees keys of its own user at or before its position
-// (M-FALCON candidates: the history and themselves), so no earlier query tile
-// and no later user's tile reads these keys.
+// Two kernels, each owning its outputs, so no gradient is accumulated with
+// atomics across CTAs:
 //
-// Tensor memory: S, then dQ, in columns [0, 128); dA in [128, 256); dK in
-// [256, 256 + HD); dV in [256 + HD, 256 + 2 HD).
+//   dq kernel   one CTA per (128-query tile, head), the query tiles in the
+//               forward's longest-first order.  Per visible key tile j:
+//                 S = Q K_j^T and dA = dO V_j^T (SS MMAs into tensor memory),
+//                 dS from S and dA (two row groups, one half of the keys each,
+//                 dS written as bf16 over the consumed S columns),
+//                 dQ += dS K_j (TS MMA: dS read from tensor memory).
+//               The row groups also sum dS into the bias-table gradients
+//               (shared-memory accumulators, one global add per entry per CTA).
+//   dkv kernel  one CTA per (128-key tile, head), longest first.  Per query
+//               tile i that can see the keys (the key tile's own tile up to the
+//               end of the user owning its last row):
+//                 S^T = K Q_i^T and dA^T = V dO_i^T (keys along the tensor-memory
+//                 lanes), P^T and dS^T from them (bf16 over the consumed columns),
+//                 dV += P^T dO_i and dK += dS^T Q_i (TS MMAs).
+//
+// Both: 12 warps.  Warp 0 issues the TMA loads (no multicast), warp 1 the MMAs
+// (one elected thread), warps 4-7 and 8-11 are two row groups; group g scores
+// columns [64 g, 64 g + 64) of every 128 x 128 tile, one tensor-memory lane
+// (row) per thread.  Tensor memory: S [0, 128), dA [128, 256), then the
+// accumulators (dQ, or dK and dV).  Every wait is bounded; a CTA that gives up
+// sets HSTU_DEVERR_TIMEOUT, drains its own copies and MMAs and frees its
+// tensor memory.
+//
+// Per (warp, half tile) the rows are classified: when every pair is visible,
+// every position bucket is the clamped one and each row meets one time bucket
+// (the common case far from the diagonal), the bias is a per-row constant and
+// the bias gradients are per-row sums; otherwise every pair takes the mask,
+// the position bucket and the exact time bucket.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -42,56 +53,36 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBwdThreads = 256;
-constexpr int kBwdMaxPos = 4097;      // pos_clamp <= 4096
+constexpr int kBwdThreads = 384;
+constexpr int kBwdMaxPos = 4097;       // pos_clamp <= 4096
 constexpr int kBwdMaxBuckets = 256;
 
-struct AttnBwdParams {
+struct BwdParams {
   const RowInfo* rows;
+  const int32_t* order;        // query-tile pairs, longest first (the forward's schedule)
+  const int32_t* key_order;    // key tiles, longest first
   const int32_t* offsets;
   int32_t B;
   const int64_t* ts;
   const int64_t* thresholds;
+  const uint8_t* time_lut;
+  const int32_t* thr32;
   const float* rab_pos;
   const float* rab_time;
   const int32_t* counters;
   int32_t* error;
-  float* dq;
-  float* dk;
-  float* dv;
   float* d_rab_pos;
   float* d_rab_time;
   int64_t T;
-  int d, H, num_key_tiles;
-  int pos_clamp, time_buckets, n_norm_fixed;
+  int d, H, num_pairs, num_key_tiles;
+  int pos_clamp, time_buckets, n_norm_fixed, lut_exact;
+  long long wait_limit;
 };
 
-template <int HD>
-struct BwdLayout {
-  static constexpr uint32_t kTile = 128 * HD * 2;                   // bf16 [128][HD]
-  static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + kTile;
-  static constexpr uint32_t kQ = kV + kTile;
-  static constexpr uint32_t kDO = kQ + kTile;
-  static constexpr uint32_t kP = kDO + kTile;                       // bf16 [128 q][128 k]
-  static constexpr uint32_t kDS = kP + 32768;
-  static constexpr uint32_t kKts = kDS + 32768;                     // int64 [128]
-  static constexpr uint32_t kThr = kKts + 1024;                     // int64 [256]
-  static constexpr uint32_t kGradTime = kThr + kBwdMaxBuckets * 8;  // float [256]
-  static constexpr uint32_t kBars = kGradTime + kBwdMaxBuckets * 4;
-  static constexpr uint32_t kGradPos = kBars + 256;                 // float [clamp + 1]
-  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
-    return kGradPos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16 + 1024;
-  }
-  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kQ % 1024 == 0 && kDO % 1024 == 0 &&
-                    kP % 1024 == 0 && kDS % 1024 == 0,
-                "swizzled tiles start on 1024-byte boundaries");
-  static_assert(kKts % 128 == 0 && kBars % 8 == 0, "alignment");
-  static_assert(smem_bytes(kBwdMaxPos - 1) <= 227 * 1024, "shared memory budget");
-};
+// ---------------------------------------------------------------- shared helpers
 
 // Largest k with thr[k] <= dt (thr[0] = 0, non-decreasing): the time bucket.
-__device__ __forceinline__ int bwd_bucket(const int64_t* thr, int nb, int64_t dt) {
+__device__ __forceinline__ int bucket_search(const int64_t* thr, int nb, int64_t dt) {
   if (dt <= 0) return 0;
   int lo = 0, hi = nb - 1;
   while (lo < hi) {
@@ -101,66 +92,175 @@ __device__ __forceinline__ int bwd_bucket(const int64_t* thr, int nb, int64_t dt
   return lo;
 }
 
-// Byte offset of column c (0..127) of row r in a [128][128] bf16 tile stored
-// as two 64-column halves of 128-byte rows with the 128-byte swizzle (16-byte
-// chunk index XOR row % 8): the layout of a TMA box of 64 x 128 bf16.
-__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
-  const int half = c >> 6;
-  const int chunk = (c & 63) >> 3;
-  return uint32_t(half * 16384 + r * 128 + ((chunk ^ (r & 7)) << 4) + (c & 7) * 2);
+// Exact time bucket of a gap and its bias.  Gaps below 2^31 - 1 with a divisor
+// whose bins are narrower than a bucket: v = dt + 1 falls in the bin
+// floor(log2 v) * 4 + (next two bits), read off v converted with truncation;
+// the bin's entry holds the next bucket's threshold and both candidate biases.
+// Anything else: a binary search of the thresholds.
+__device__ __forceinline__ int time_bucket(int64_t dt, bool lut, const int4* s_any,
+                                           const int64_t* s_thr, const float* s_rt, int nb,
+                                           float& rt) {
+  if (dt < 0) dt = 0;
+  if (lut && dt < int64_t(0x7FFFFFFE)) {
+    const uint32_t v = uint32_t(dt) + 1u;
+    const uint32_t fb = __float_as_uint(__uint2float_rz(v));
+    const int4 e = s_any[int((fb >> 21) - 508u) & 127];
+    const bool up = int(dt) >= e.x;
+    rt = __int_as_float(up ? e.z : e.y);
+    return e.w + (up ? 1 : 0);
+  }
+  const int b = bucket_search(s_thr, nb, dt);
+  rt = s_rt[b];
+  return b;
 }
+
+// The per-CTA tables, written by the 256 row-group threads (t = 0..255).
+__device__ __forceinline__ void load_tables(const BwdParams& p, int t, int64_t* s_thr, float* s_rt,
+                                            int4* s_any) {
+  const int nb = p.time_buckets;
+  s_thr[t] = t < nb ? __ldg(p.thresholds + t) : (int64_t(1) << 62);
+  s_rt[t] = t < nb ? __ldg(p.rab_time + t) : 0.0f;
+  if (t < 128) {
+    const int cand = __ldg(p.time_lut + t);
+    const int nxt = cand + 1 < nb ? cand + 1 : cand;
+    s_any[t] = make_int4(cand + 1 < nb ? __ldg(p.thr32 + cand + 1) : 0x7FFFFFFF,
+                         __float_as_int(__ldg(p.rab_time + cand)),
+                         __float_as_int(__ldg(p.rab_time + nxt)), cand);
+  }
+}
+
+// sig(s) / n_norm (pre-scaled) and the two results of one pair.
+struct Grad {
+  float p;    // SiLU(s) / n_norm
+  float ds;   // dA SiLU'(s) / n_norm
+};
+__device__ __forceinline__ Grad silu_grad(float s, float da, float inv_nn) {
+  const float sig = fmaf(0.5f, tanh_approx(0.5f * s), 0.5f);
+  const float sn = sig * inv_nn;
+  const float w = fmaf(s, 1.0f - sig, 1.0f);
+  Grad g;
+  g.p = s * sn;
+  g.ds = da * (sn * w);
+  return g;
+}
+
+// Tensor-memory column of the bf16 operand (P or dS) for K-step kk of a TS MMA:
+// group g writes its keys' packed pairs over the first half of its own 64
+// score columns.
+__device__ __forceinline__ uint32_t a_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Stages 32 rows x 32 fp32 columns of tensor memory (this warp's lanes) into a
+// 128-byte-swizzled 4 KB box and writes it with a TMA store at (x, y).
+__device__ __forceinline__ void store_box(uint32_t taddr, uint8_t* box, const CUtensorMap* m,
+                                          int32_t x, int32_t y, int lane) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_ld_wait();
+  const uint32_t row_addr = smem_u32(box + lane * 128);
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4), __uint_as_float(r[4 * e + 0]),
+                 __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                 __uint_as_float(r[4 * e + 3]));
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(m, box, x, y);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+}
+
+// ================================================================ dq kernel
+
+template <int HD>
+struct DqLayout {
+  static constexpr int NS = HD == 128 ? 2 : 3;    // K / V ring stages
+  static constexpr uint32_t kTile = 128 * HD * 2;
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kDO = kTile;
+  static constexpr uint32_t kK = 2 * kTile;
+  static constexpr uint32_t kV = kK + NS * kTile;
+  static constexpr uint32_t kKts = kV + NS * kTile;         // int64 [NS][128]
+  static constexpr uint32_t kThr = kKts + NS * 1024;        // int64 [256]
+  static constexpr uint32_t kRt = kThr + 2048;              // float [256]
+  static constexpr uint32_t kGtime = kRt + 1024;            // float [256]
+  static constexpr uint32_t kAny = kGtime + 1024;           // int4 [128]
+  static constexpr uint32_t kBars = kAny + 2048;
+  static constexpr uint32_t kGpos = kBars + 256;            // float [clamp + 1]
+  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
+    return kGpos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16 + 1024;
+  }
+  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kTile % 1024 == 0, "tile alignment");
+  static_assert(kKts % 128 == 0 && kBars % 8 == 0 && kAny % 16 == 0, "alignment");
+  // dQ is staged in the Q and dO tiles: 8 warps x HD / 64 boxes of 4 KB
+  static_assert(8 * (HD / 64) * 4096 == 2 * kTile, "dQ staging");
+  static_assert(smem_bytes(kBwdMaxPos - 1) <= 227 * 1024, "shared memory budget");
+};
 
 template <int HD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_ts, const AttnBwdParams p) {
-  using L = BwdLayout<HD>;
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_ts,
+                       const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using L = DqLayout<HD>;
+  constexpr int NS = L::NS;
+  // ---- work item: one query tile of the pair order, one head
+  const int per_head = 2 * p.num_pairs;
+  const int h = blockIdx.x / per_head;
+  const int rr = blockIdx.x % per_head;
+  const int qt = 2 * p.order[rr >> 1] + (rr & 1);
+  const int64_t r0 = int64_t(qt) * 128;
+  if (r0 >= p.T) return;   // the missing second tile of the last pair (uniform over the CTA)
+  int a0, e0;
+  range_before(p.rows, r0, a0, e0);
+  const int a_hi = e0 < qt ? (e0 > a0 ? e0 : a0) : qt;
+  const int n_a = a_hi - a0;
+  const int n_kt = n_a + 1;
+  auto key_tile = [&](int j) -> int { return j < n_a ? a0 + j : qt; };
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int64_t* s_kts = reinterpret_cast<int64_t*>(smem + L::kKts);
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
-  float* s_gtime = reinterpret_cast<float*>(smem + L::kGradTime);
-  float* s_gpos = reinterpret_cast<float*>(smem + L::kGradPos);
+  float* s_rt = reinterpret_cast<float*>(smem + L::kRt);
+  float* s_gtime = reinterpret_cast<float*>(smem + L::kGtime);
+  int4* s_any = reinterpret_cast<int4*>(smem + L::kAny);
+  float* s_gpos = reinterpret_cast<float*>(smem + L::kGpos);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* kv_full = bars;         // K, V, key timestamps landed
-  uint64_t* q_full = bars + 1;      // Q and dO of the current query tile landed
-  uint64_t* q_empty = bars + 2;     // every MMA reading Q and dO is done
-  uint64_t* s_full = bars + 3;      // S and dA are in tensor memory
-  uint64_t* p_full = bars + 4;      // P and dS are in shared memory (128 arrivals)
-  uint64_t* mma_done = bars + 5;    // dV, dK, dQ products of the tile are done
-  uint64_t* tmem_free = bars + 6;   // dQ read out: S / dA columns free (128 arrivals)
-  uint64_t* kv_done = bars + 7;     // every product of the CTA is done
-  uint64_t* drained = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = q_full + 1;      // [NS]
+  uint64_t* kv_empty = kv_full + NS;   // [NS]
+  uint64_t* s_full = kv_empty + NS;    // S and dA of the current key tile are in tensor memory
+  uint64_t* ds_full = s_full + 1;      // dS written (256 arrivals)
+  uint64_t* dq_done = ds_full + 1;     // every product is done
+  uint64_t* drained = dq_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int d = p.d;
-  const int kt = blockIdx.x % p.num_key_tiles;
-  const int h = blockIdx.x / p.num_key_tiles;
-  const int64_t kb = int64_t(kt) * 128;
-
-  // the query tiles that read this key tile: [kt, end of the last row's user)
-  int64_t r_last = kb + 127 < p.T ? kb + 127 : p.T - 1;
-  int32_t u = p.rows[r_last].user;
-  u = u < 0 ? 0 : (u >= p.B ? p.B - 1 : u);
-  int64_t ue = p.offsets[u + 1];
-  if (ue <= r_last) ue = r_last + 1;
-  if (ue > p.T) ue = p.T;
-  const int q_begin = kt;
-  const int nq = int((ue + 127) / 128) - q_begin;   // >= 1
+  const int clamp = p.pos_clamp;
+  const int nb = p.time_buckets;
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(mma_done, 1);
-    mbar_init(tmem_free, 128);
-    mbar_init(kv_done, 1);
+    mbar_init(ds_full, 256);
+    mbar_init(dq_done, 1);
     mbar_init(drained, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -169,22 +269,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // the tables and the gradient accumulators
-  const int clamp = p.pos_clamp;
-  const int nb = p.time_buckets;
-  for (int k = threadIdx.x; k < kBwdMaxBuckets; k += blockDim.x) {
-    s_thr[k] = k < nb ? p.thresholds[k] : (int64_t(1) << 62);
-    s_gtime[k] = 0.0f;
+  if (warp >= 4) {
+    const int t = threadIdx.x - 128;
+    load_tables(p, t, s_thr, s_rt, s_any);
+    s_gtime[t] = 0.0f;
+    for (int k = t; k <= clamp; k += 256) s_gpos[k] = 0.0f;
   }
-  for (int k = threadIdx.x; k <= clamp; k += blockDim.x) s_gpos[k] = 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tS = tmem_base;
   const uint32_t tdA = tmem_base + 128;
-  const uint32_t tdK = tmem_base + 256;
-  const uint32_t tdV = tmem_base + 256 + HD;
+  const uint32_t tDQ = tmem_base + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
@@ -192,238 +289,232 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       prefetch_tmap(&tm);
       prefetch_tmap(&tm_do);
       prefetch_tmap(&tm_ts);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kTile + 128 * 8);
+      mbar_arrive_expect_tx(q_full, 2 * L::kTile);
 #pragma unroll
       for (int b = 0; b < HD / 64; ++b) {
-        tma_load_2d(smem + L::kK + b * 16384, &tm, kv_full, 3 * d + h * HD + b * 64, int32_t(kb));
-        tma_load_2d(smem + L::kV + b * 16384, &tm, kv_full, d + h * HD + b * 64, int32_t(kb));
+        tma_load_2d(smem + L::kQ + b * 16384, &tm, q_full, 2 * d + h * HD + b * 64, int32_t(r0));
+        tma_load_2d(smem + L::kDO + b * 16384, &tm_do, q_full, h * HD + b * 64, int32_t(r0));
       }
-      tma_load_1d(s_kts, &tm_ts, kv_full, int32_t(kb));
-      int issued = 0;
-      for (int it = 0; it < nq && !*abort_flag; ++it) {
-        if (it > 0 && !mbar_wait(q_empty, (it - 1) & 1)) { *abort_flag = 1; break; }
-        const int32_t row0 = (q_begin + it) * 128;
-        mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+      bool issued[NS];
+      uint32_t issued_ph[NS];
+      for (int s = 0; s < NS; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int s = j % NS;
+        const uint32_t ph = (j / NS) & 1;
+        if (!mbar_wait(&kv_empty[s], ph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
+        const int32_t kb = key_tile(j) * 128;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * L::kTile + 1024);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b) {
-          tma_load_2d(smem + L::kQ + b * 16384, &tm, q_full, 2 * d + h * HD + b * 64, row0);
-          tma_load_2d(smem + L::kDO + b * 16384, &tm_do, q_full, h * HD + b * 64, row0);
+          tma_load_2d(smem + L::kK + s * L::kTile + b * 16384, &tm, &kv_full[s],
+                      3 * d + h * HD + b * 64, kb);
+          tma_load_2d(smem + L::kV + s * L::kTile + b * 16384, &tm, &kv_full[s],
+                      d + h * HD + b * 64, kb);
         }
-        issued = it + 1;
+        tma_load_1d(s_kts + s * 128, &tm_ts, &kv_full[s], kb);
+        issued[s] = true;
+        issued_ph[s] = ph;
       }
       // no copy may still be in flight when the CTA ends
-      mbar_wait(kv_full, 0);
-      if (issued > 0) mbar_wait(q_full, (issued - 1) & 1);
+      mbar_wait(q_full, 0);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s]) mbar_wait(&kv_full[s], issued_ph[s]);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);   // S, dA
-      constexpr uint32_t idesc_t = idesc_bf16(128, HD, true, true);       // dV, dK
-      constexpr uint32_t idesc_q = idesc_bf16(128, HD, false, true);      // dQ
-      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);   // S, dA
+      constexpr uint32_t idesc_dq = idesc_bf16(128, HD, false, true);     // dQ
       const uint32_t sQ = smem_u32(smem + L::kQ), sDO = smem_u32(smem + L::kDO);
-      const uint32_t sP = smem_u32(smem + L::kP), sDS = smem_u32(smem + L::kDS);
-      bool ok = mbar_wait(kv_full, 0);
-      for (int it = 0; ok && it < nq; ++it) {
-        if (!mbar_wait(q_full, it & 1)) { ok = false; break; }
-        if (it > 0 && !mbar_wait(tmem_free, (it - 1) & 1)) { ok = false; break; }
+      bool ok = mbar_wait(q_full, 0, p.wait_limit);
+      for (int j = 0; ok && j < n_kt; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(&kv_full[s], (j / NS) & 1, p.wait_limit)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t sK = smem_u32(smem + L::kK + s * L::kTile);
+        const uint32_t sV = smem_u32(smem + L::kV + s * L::kTile);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tS, desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024), idesc_kk,
+          umma_ss(tS, desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024), idesc_ss,
                   kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tdA, desc_sw128(sDO + off, 16, 1024), desc_sw128(sV + off, 16, 1024), idesc_kk,
+          umma_ss(tdA, desc_sw128(sDO + off, 16, 1024), desc_sw128(sV + off, 16, 1024), idesc_ss,
                   kk > 0);
         }
         umma_commit(s_full);
-        if (!mbar_wait(p_full, it & 1)) { ok = false; break; }
+        if (!mbar_wait(ds_full, j & 1, p.wait_limit)) { ok = false; break; }
         tc_fence_after();
-        // K = the 128 query rows, in 8 steps of 16 (2048 bytes of 128-byte rows)
+        // dQ += dS K_j: K = the 128 keys in 8 steps of 16, K_j consumed N-major
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_ss(tdV, desc_sw128(sP + kk * 2048, 16384, 1024),
-                  desc_sw128(sDO + kk * 2048, 16384, 1024), idesc_t, (it > 0 || kk > 0));
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_ss(tdK, desc_sw128(sDS + kk * 2048, 16384, 1024),
-                  desc_sw128(sQ + kk * 2048, 16384, 1024), idesc_t, (it > 0 || kk > 0));
-        }
-        umma_commit(q_empty);
-        // K = the 128 keys: dS K-major (two 64-key halves), K N-major
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tS, desc_sw128(sDS + off, 16, 1024), desc_sw128(sK + kk * 2048, 16384, 1024),
-                  idesc_q, kk > 0);
-        }
-        umma_commit(mma_done);
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDQ, tS + a_col(kk), desc_sw128(sK + kk * 2048, 16384, 1024), idesc_dq,
+                  (j > 0 || kk > 0));
+        umma_commit(&kv_empty[s]);
       }
       if (!ok) *abort_flag = 1;
-      umma_commit(kv_done);     // releases the final read-out (also on an abort)
+      umma_commit(dq_done);      // also releases the read-out after an abort
       umma_commit(drained);
       mbar_wait(drained, 0);
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ rows
-    const int wq = warp & 3;
+    // ------------------------------------------------------------ row groups
+    const int g = (warp - 4) >> 2;           // key half of every tile
+    const int wq = warp & 3;                 // tensor-memory lane quarter
     const int row = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const int64_t i = r0 + row;
+    const bool valid = i < p.T;
+    int lo = 0, hi = 0, pos = 0;
+    int64_t ti = 0;
+    if (valid) {
+      const RowInfo ri = p.rows[i];
+      lo = (ri.lo < 0 || ri.lo > i) ? int(i) : ri.lo;
+      hi = ri.hi;
+      pos = ri.pos;
+      ti = p.ts[i];
+    }
     const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
-    bool ok = mbar_wait(kv_full, 0);
-    ok = __all_sync(0xffffffffu, ok);
-    uint8_t* sP = smem + L::kP;
-    uint8_t* sDS = smem + L::kDS;
-    for (int it = 0; ok && it < nq; ++it) {
-      const int64_t i = int64_t(q_begin + it) * 128 + row;
-      const bool valid = i < p.T;
-      int64_t lo = i, hi = i, pos = i, ti = 0;
-      if (valid) {
-        const RowInfo ri = p.rows[i];
-        lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
-        hi = ri.hi;
-        pos = ri.pos;
-        ti = p.ts[i];
+    const bool lut = p.lut_exact != 0;
+    const float rp_clamp = __ldg(p.rab_pos + clamp);
+    named_bar_sync(1, 256);   // the tables
+    bool aborted = false;
+    for (int j = 0; j < n_kt; ++j) {
+      const int s = j % NS;
+      const int kb = key_tile(j) * 128;
+      bool ok = aborted ? false : mbar_wait(&kv_full[s], (j / NS) & 1, p.wait_limit);
+      ok = ok && mbar_wait(s_full, j & 1, p.wait_limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        aborted = true;
+        *abort_flag = 1;
+        break;
       }
-      bool w = mbar_wait(s_full, it & 1);
-      w = __all_sync(0xffffffffu, w);
-      if (!w) { ok = false; break; }
       tc_fence_after();
-      bool any = false;
-      // Along a row the keys advance in time inside the user, so the gap only
-      // shrinks: the time bucket walks down from the previous visible key's (a
-      // larger gap, i.e. input out of order, searches again).  The bias
-      // gradients are summed in registers while the bucket stays the same
-      // (time) or for the clamped entry (position), and added to shared
-      // memory when the bucket changes and at the end of the tile.
-      int tb = -1;
-      float acc_t = 0.0f, acc_c = 0.0f;
+      const int64_t* kts = s_kts + s * 128;
+      const int j0 = kb + 64 * g;   // first key of this group's half
+      // ---- classify the row for this half tile
+      const bool zero = __all_sync(0xffffffffu, !valid || i < j0);
+      const bool full = valid && lo <= j0 && j0 + 63 < hi;
+      int tb0 = 0;
+      bool same = false;
+      if (full) {
+        tb0 = bucket_search(s_thr, nb, ti - kts[64 * g]);
+        same = tb0 == bucket_search(s_thr, nb, ti - kts[64 * g + 63]);
+      }
+      const bool fast = __all_sync(0xffffffffu, full && same && pos - (j0 + 63) >= clamp);
+      const uint32_t tcol = lane_off + 64 * g;
+      if (zero) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[e] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st8(tS + tcol + 8 * c, pk);
+      } else if (fast) {
+        // every pair visible, clamped position, one time bucket per row
+        const float hc = rp_clamp + s_rt[tb0];
+        float acc = 0.0f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t rs[32], ra[32];
-        tmem_ld32(tS + lane_off + c0, rs);
-        tmem_ld32(tdA + lane_off + c0, ra);
-        tmem_ld_wait();
-        uint32_t pa[16], pd[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pk[8];
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float av[2], dv[2];
+          for (int e = 0; e < 16; e += 2) {
+            const Grad g0 = silu_grad(__uint_as_float(rs[e]) + hc, __uint_as_float(ra[e]), inv_nn);
+            const Grad g1 =
+                silu_grad(__uint_as_float(rs[e + 1]) + hc, __uint_as_float(ra[e + 1]), inv_nn);
+            acc += g0.ds + g1.ds;
+            pk[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+          }
+          tmem_st8(tS + tcol + 8 * c, pk);
+        }
+        // the position bucket is the clamped one for the whole warp
+        const float wsum = warp_sum(acc);
+        if (lane == 0 && wsum != 0.0f) atomicAdd(s_gpos + clamp, wsum);
+        if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
+          if (lane == 0 && wsum != 0.0f) atomicAdd(s_gtime + tb0, wsum);
+        } else if (acc != 0.0f) {
+          atomicAdd(s_gtime + tb0, acc);
+        }
+      } else {
+        // any visibility: the mask, the position bucket and the exact time bucket
+        // of every pair; bias gradients summed along runs of one bucket
+        int run_b = -1;
+        float run_acc = 0.0f, acc_c = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pk[8];
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
+          float dsv[16];
 #pragma unroll
-          for (int f = 0; f < 2; ++f) {
-            const int c = c0 + e + f;
-            const int64_t j = kb + c;
-            const bool vis = valid && j < p.T && ((lo <= j && j < hi) || j == i);
-            av[f] = 0.0f;
-            dv[f] = 0.0f;
+          for (int e = 0; e < 16; ++e) {
+            const int jr = 64 * g + 16 * c + e;
+            const int jj = kb + jr;
+            const bool vis = valid && jj < p.T && ((lo <= jj && jj < hi) || int64_t(jj) == i);
+            float rt;
+            const int tb = time_bucket(ti - kts[jr], lut, s_any, s_thr, s_rt, nb, rt);
+            int dp = pos - jj;
+            dp = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+            const float sc = __uint_as_float(rs[e]) + __ldg(p.rab_pos + dp) + rt;
+            const Grad gr = silu_grad(sc, __uint_as_float(ra[e]), inv_nn);
+            const float ds = vis ? gr.ds : 0.0f;
+            dsv[e] = ds;
             if (vis) {
-              int64_t rel = pos - j;
-              const int pidx = rel < 0 ? 0 : (rel > clamp ? clamp : int(rel));
-              const int64_t gap = ti - s_kts[c];
-              int tidx;
-              if (tb < 0 || (tb + 1 < nb && gap >= s_thr[tb + 1])) {
-                tidx = bwd_bucket(s_thr, nb, gap);
-              } else {
-                tidx = tb;
-                while (tidx > 0 && gap < s_thr[tidx]) --tidx;
+              if (dp == clamp) acc_c += ds;
+              else atomicAdd(s_gpos + dp, ds);
+              if (tb != run_b) {
+                if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
+                run_b = tb;
+                run_acc = 0.0f;
               }
-              const float s = __uint_as_float(rs[e + f]) + __ldg(p.rab_pos + pidx) +
-                              __ldg(p.rab_time + tidx);
-              const float sig = 0.5f + 0.5f * tanh_approx(0.5f * s);
-              av[f] = s * sig * inv_nn;
-              const float ds = __uint_as_float(ra[e + f]) * (sig * (1.0f + s * (1.0f - sig))) * inv_nn;
-              dv[f] = ds;
-              if (pidx == clamp) acc_c += ds;
-              else atomicAdd(s_gpos + pidx, ds);
-              if (tidx != tb) {
-                if (tb >= 0 && acc_t != 0.0f) atomicAdd(s_gtime + tb, acc_t);
-                tb = tidx;
-                acc_t = 0.0f;
-              }
-              acc_t += ds;
-              any = true;
+              run_acc += ds;
             }
           }
-          pa[e / 2] = pack_bf16x2(av[0], av[1]);
-          pd[e / 2] = pack_bf16x2(dv[0], dv[1]);
-        }
-        // 32 columns = four 16-byte chunks of P and of dS
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t off = sw128_offset(row, c0 + g * 8);
-          st_shared_v4_u32(smem_u32(sP + off), pa[4 * g], pa[4 * g + 1], pa[4 * g + 2], pa[4 * g + 3]);
-          st_shared_v4_u32(smem_u32(sDS + off), pd[4 * g], pd[4 * g + 1], pd[4 * g + 2], pd[4 * g + 3]);
+          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
+          tmem_st8(tS + tcol + 8 * c, pk);
         }
+        if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
+        if (acc_c != 0.0f) atomicAdd(s_gpos + clamp, acc_c);
       }
-      if (tb >= 0 && acc_t != 0.0f) atomicAdd(s_gtime + tb, acc_t);
-      if (acc_c != 0.0f) atomicAdd(s_gpos + clamp, acc_c);
-      fence_proxy_async_smem();   // the tensor cores read P and dS through the async proxy
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
-      w = mbar_wait(mma_done, it & 1);
-      w = __all_sync(0xffffffffu, w);
-      if (!w) { ok = false; break; }
-      tc_fence_after();
-      // dQ of this (query tile, key tile) into the global fp32 accumulator
-      const bool add = __any_sync(0xffffffffu, any);
-#pragma unroll 1
-      for (int c0 = 0; add && c0 < HD; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + c0, r);
-        tmem_ld_wait();
-        if (any) {
-          float* dst = p.dq + i * d + h * HD + c0;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) atomicAdd(dst + e, __uint_as_float(r[e]));
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(tmem_free);
+      mbar_arrive(ds_full);
     }
-    if (!ok) *abort_flag = 1;
-    // dK and dV of the key tile: one key row per thread
-    bool w = ok ? mbar_wait(kv_done, 0) : false;
+    if (aborted) *abort_flag = 1;
+    // ---- dQ -> the (now free) Q and dO tiles -> TMA stores; the rows past T are clipped
+    bool w = aborted ? false : mbar_wait(dq_done, 0, p.wait_limit);
     w = __all_sync(0xffffffffu, w);
-    if (w) {
+    if (w && !*abort_flag) {
       tc_fence_after();
-      const int64_t j = kb + row;
+      uint8_t* stage = smem + L::kQ + (g * 4 + wq) * (HD / 64) * 4096;
 #pragma unroll 1
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t rk[32], rv[32];
-        tmem_ld32(tdK + lane_off + c0, rk);
-        tmem_ld32(tdV + lane_off + c0, rv);
-        tmem_ld_wait();
-        if (j < p.T) {
-          float4* gk = reinterpret_cast<float4*>(p.dk + j * d + h * HD + c0);
-          float4* gv = reinterpret_cast<float4*>(p.dv + j * d + h * HD + c0);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            gk[e] = make_float4(__uint_as_float(rk[4 * e]), __uint_as_float(rk[4 * e + 1]),
-                                __uint_as_float(rk[4 * e + 2]), __uint_as_float(rk[4 * e + 3]));
-            gv[e] = make_float4(__uint_as_float(rv[4 * e]), __uint_as_float(rv[4 * e + 1]),
-                                __uint_as_float(rv[4 * e + 2]), __uint_as_float(rv[4 * e + 3]));
-          }
-        }
+      for (int cb = 0; cb < HD / 64; ++cb) {
+        const int col = g * (HD / 2) + cb * 32;
+        store_box(tDQ + lane_off + col, stage + cb * 4096, &tm_dq, h * HD + col,
+                  int32_t(r0) + wq * 32, lane);
       }
     } else {
       *abort_flag = 1;
     }
-    // the bias gradients of the CTA
-    named_bar_sync(1, 128);
+    // ---- the bias gradients of the CTA
+    named_bar_sync(1, 256);
     const int t = threadIdx.x - 128;
-    for (int k = t; k <= clamp; k += 128) {
-      const float g = s_gpos[k];
-      if (g != 0.0f) atomicAdd(p.d_rab_pos + k, g);
+    for (int k = t; k <= clamp; k += 256) {
+      const float gv = s_gpos[k];
+      if (gv != 0.0f) atomicAdd(p.d_rab_pos + k, gv);
     }
-    for (int k = t; k < nb; k += 128) {
-      const float g = s_gtime[k];
-      if (g != 0.0f) atomicAdd(p.d_rab_time + k, g);
+    if (t < nb) {
+      const float gv = s_gtime[t];
+      if (gv != 0.0f) atomicAdd(p.d_rab_time + t, gv);
     }
   }
 
@@ -436,47 +527,419 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ================================================================ dkv kernel
+
+template <int HD>
+struct DkvLayout {
+  static constexpr int NS = HD == 128 ? 2 : 3;    // Q / dO ring stages
+  static constexpr uint32_t kTile = 128 * HD * 2;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kTile;
+  static constexpr uint32_t kQ = 2 * kTile;
+  static constexpr uint32_t kDO = kQ + NS * kTile;
+  static constexpr uint32_t kQf = kDO + NS * kTile;          // RowInfo [NS][128]
+  static constexpr uint32_t kQts = kQf + NS * 2048;          // int64 [NS][128]
+  static constexpr uint32_t kThr = kQts + NS * 1024;         // int64 [256]
+  static constexpr uint32_t kRt = kThr + 2048;               // float [256]
+  static constexpr uint32_t kAny = kRt + 1024;               // int4 [128]
+  static constexpr uint32_t kBars = kAny + 2048;
+  static constexpr uint32_t kSmemBytes = kBars + 256 + 1024;
+  static_assert(kQ % 1024 == 0 && kDO % 1024 == 0 && kTile % 1024 == 0, "tile alignment");
+  static_assert(kQf % 128 == 0 && kQts % 128 == 0 && kAny % 16 == 0, "alignment");
+  // dK / dV are staged in the K and V tiles: 8 warps x HD / 64 boxes per pass, two passes
+  static_assert(8 * (HD / 64) * 4096 == 2 * kTile, "dK / dV staging");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int HD>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_ts,
+                        const __grid_constant__ CUtensorMap tm_rows,
+                        const __grid_constant__ CUtensorMap tm_dk,
+                        const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+  using L = DkvLayout<HD>;
+  constexpr int NS = L::NS;
+  // ---- work item: one key tile (longest first), one head
+  const int h = blockIdx.x / p.num_key_tiles;
+  const int kt = p.key_order[blockIdx.x % p.num_key_tiles];
+  const int64_t kb = int64_t(kt) * 128;
+  // the query tiles that can see these keys: [kt, end of the user owning the last key)
+  const int64_t r_last = kb + 127 < p.T ? kb + 127 : p.T - 1;
+  int32_t u = p.rows[r_last].user;
+  u = u < 0 ? 0 : (u >= p.B ? p.B - 1 : u);
+  int64_t ue = p.offsets[u + 1];
+  if (ue <= r_last) ue = r_last + 1;
+  if (ue > p.T) ue = p.T;
+  const int nq = int((ue + 127) / 128) - kt;   // >= 1
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const RowInfo* s_qf = reinterpret_cast<const RowInfo*>(smem + L::kQf);
+  const int64_t* s_qts = reinterpret_cast<const int64_t*>(smem + L::kQts);
+  int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
+  float* s_rt = reinterpret_cast<float*>(smem + L::kRt);
+  int4* s_any = reinterpret_cast<int4*>(smem + L::kAny);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = kv_full + 1;      // [NS] Q, dO and the query facts of a tile landed
+  uint64_t* q_empty = q_full + NS;     // [NS]
+  uint64_t* s_full = q_empty + NS;     // S^T and dA^T are in tensor memory
+  uint64_t* p_full = s_full + 1;       // P^T and dS^T written (256 arrivals)
+  uint64_t* kv_done = p_full + 1;      // every product is done
+  uint64_t* drained = kv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int d = p.d;
+  const int clamp = p.pos_clamp;
+  const int nb = p.time_buckets;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(kv_done, 1);
+    mbar_init(drained, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp >= 4) load_tables(p, threadIdx.x - 128, s_thr, s_rt, s_any);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tS = tmem_base;
+  const uint32_t tdA = tmem_base + 128;
+  const uint32_t tDK = tmem_base + 256;
+  const uint32_t tDV = tmem_base + 256 + HD;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      prefetch_tmap(&tm);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_ts);
+      prefetch_tmap(&tm_rows);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
+#pragma unroll
+      for (int b = 0; b < HD / 64; ++b) {
+        tma_load_2d(smem + L::kK + b * 16384, &tm, kv_full, 3 * d + h * HD + b * 64, int32_t(kb));
+        tma_load_2d(smem + L::kV + b * 16384, &tm, kv_full, d + h * HD + b * 64, int32_t(kb));
+      }
+      bool issued[NS];
+      uint32_t issued_ph[NS];
+      for (int s = 0; s < NS; ++s) issued[s] = false, issued_ph[s] = 0;
+      for (int it = 0; it < nq && !*abort_flag; ++it) {
+        const int s = it % NS;
+        const uint32_t ph = (it / NS) & 1;
+        if (!mbar_wait(&q_empty[s], ph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
+        const int32_t q0 = (kt + it) * 128;
+        mbar_arrive_expect_tx(&q_full[s], 2 * L::kTile + 2048 + 1024);
+#pragma unroll
+        for (int b = 0; b < HD / 64; ++b) {
+          tma_load_2d(smem + L::kQ + s * L::kTile + b * 16384, &tm, &q_full[s],
+                      2 * d + h * HD + b * 64, q0);
+          tma_load_2d(smem + L::kDO + s * L::kTile + b * 16384, &tm_do, &q_full[s],
+                      h * HD + b * 64, q0);
+        }
+        // the query rows' facts (RowInfo as pairs of int64) and timestamps
+        tma_load_1d(smem + L::kQf + s * 2048, &tm_rows, &q_full[s], 2 * q0);
+        tma_load_1d(smem + L::kQts + s * 1024, &tm_ts, &q_full[s], q0);
+        issued[s] = true;
+        issued_ph[s] = ph;
+      }
+      mbar_wait(kv_full, 0);
+      for (int s = 0; s < NS; ++s)
+        if (issued[s]) mbar_wait(&q_full[s], issued_ph[s]);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16(128, 128, false, false);   // S^T, dA^T
+      constexpr uint32_t idesc_kv = idesc_bf16(128, HD, false, true);     // dV, dK
+      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      bool ok = mbar_wait(kv_full, 0, p.wait_limit);
+      for (int it = 0; ok && it < nq; ++it) {
+        const int s = it % NS;
+        if (!mbar_wait(&q_full[s], (it / NS) & 1, p.wait_limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(smem + L::kQ + s * L::kTile);
+        const uint32_t sDO = smem_u32(smem + L::kDO + s * L::kTile);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tS, desc_sw128(sK + off, 16, 1024), desc_sw128(sQ + off, 16, 1024), idesc_ss,
+                  kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tdA, desc_sw128(sV + off, 16, 1024), desc_sw128(sDO + off, 16, 1024), idesc_ss,
+                  kk > 0);
+        }
+        umma_commit(s_full);
+        if (!mbar_wait(p_full, it & 1, p.wait_limit)) { ok = false; break; }
+        tc_fence_after();
+        // K = the 128 queries in 8 steps of 16; dO_i and Q_i consumed N-major
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDV, tS + a_col(kk), desc_sw128(sDO + kk * 2048, 16384, 1024), idesc_kv,
+                  (it > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDK, tdA + a_col(kk), desc_sw128(sQ + kk * 2048, 16384, 1024), idesc_kv,
+                  (it > 0 || kk > 0));
+        umma_commit(&q_empty[s]);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(kv_done);
+      umma_commit(drained);
+      mbar_wait(drained, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ row groups (rows = keys)
+    const int g = (warp - 4) >> 2;           // query half of every tile
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const int64_t jk = kb + row;             // this thread's key
+    const bool valid = jk < p.T;
+    const int j = int(jk);
+    const int64_t tj = valid ? p.ts[jk] : 0;
+    const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
+    const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
+    const bool lut = p.lut_exact != 0;
+    const float rp_clamp = __ldg(p.rab_pos + clamp);
+    named_bar_sync(1, 256);   // the tables
+    bool aborted = false;
+    for (int it = 0; it < nq; ++it) {
+      const int s = it % NS;
+      const int64_t q0 = int64_t(kt + it) * 128;
+      bool ok = aborted ? false : mbar_wait(&q_full[s], (it / NS) & 1, p.wait_limit);
+      ok = ok && mbar_wait(s_full, it & 1, p.wait_limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        aborted = true;
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const RowInfo* qf = s_qf + s * 128;
+      const int64_t* qts = s_qts + s * 128;
+      const int64_t i0 = q0 + 64 * g;   // first query of this group's half
+      // ---- classify the key row for this half tile: the half's queries' facts,
+      // reduced over the warp (each lane reads two)
+      int mx_lo, mn_hi, mn_pos;
+      {
+        const RowInfo fa = qf[64 * g + lane], fb = qf[64 * g + 32 + lane];
+        mx_lo = max(fa.lo, fb.lo);
+        mn_hi = min(fa.hi, fb.hi);
+        mn_pos = min(fa.pos, fb.pos);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          mx_lo = max(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, o));
+          mn_hi = min(mn_hi, __shfl_xor_sync(0xffffffffu, mn_hi, o));
+          mn_pos = min(mn_pos, __shfl_xor_sync(0xffffffffu, mn_pos, o));
+        }
+      }
+      const bool all_rows = i0 + 63 < p.T;
+      const bool zero = __all_sync(0xffffffffu, !valid || i0 + 63 < jk);
+      const bool full = valid && all_rows && mx_lo <= j && j < mn_hi;
+      int tb0 = 0;
+      bool same = false;
+      if (full) {
+        tb0 = bucket_search(s_thr, nb, qts[64 * g] - tj);
+        same = tb0 == bucket_search(s_thr, nb, qts[64 * g + 63] - tj);
+      }
+      const bool fast = __all_sync(0xffffffffu, full && same && mn_pos - j >= clamp);
+      const uint32_t tcol = lane_off + 64 * g;
+      if (zero) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[e] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_st8(tS + tcol + 8 * c, pk);
+          tmem_st8(tdA + tcol + 8 * c, pk);
+        }
+      } else if (fast) {
+        const float hc = rp_clamp + s_rt[tb0];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pp[8], pd[8];
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const Grad g0 = silu_grad(__uint_as_float(rs[e]) + hc, __uint_as_float(ra[e]), inv_nn);
+            const Grad g1 =
+                silu_grad(__uint_as_float(rs[e + 1]) + hc, __uint_as_float(ra[e + 1]), inv_nn);
+            pp[e >> 1] = pack_bf16x2(g0.p, g1.p);
+            pd[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+          }
+          tmem_st8(tS + tcol + 8 * c, pp);
+          tmem_st8(tdA + tcol + 8 * c, pd);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pp[8], pd[8];
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
+          float pv[16], dv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int ir = 64 * g + 16 * c + e;
+            const int64_t iq = q0 + ir;
+            const RowInfo f = qf[ir];
+            const bool vis = valid && iq < p.T && ((f.lo <= j && j < f.hi) || iq == jk);
+            float rt;
+            time_bucket(qts[ir] - tj, lut, s_any, s_thr, s_rt, nb, rt);
+            int dp = f.pos - j;
+            dp = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+            const float sc = __uint_as_float(rs[e]) + __ldg(p.rab_pos + dp) + rt;
+            const Grad gr = silu_grad(sc, __uint_as_float(ra[e]), inv_nn);
+            pv[e] = vis ? gr.p : 0.0f;
+            dv[e] = vis ? gr.ds : 0.0f;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pp[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+            pd[e] = pack_bf16x2(dv[2 * e], dv[2 * e + 1]);
+          }
+          tmem_st8(tS + tcol + 8 * c, pp);
+          tmem_st8(tdA + tcol + 8 * c, pd);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (aborted) *abort_flag = 1;
+    // ---- dK (group 0) / dV (group 1) -> the free K and V tiles -> TMA stores
+    bool w = aborted ? false : mbar_wait(kv_done, 0, p.wait_limit);
+    w = __all_sync(0xffffffffu, w);
+    if (w && !*abort_flag) {
+      tc_fence_after();
+      const uint32_t tacc = g == 0 ? tDK : tDV;
+      const CUtensorMap* m = g == 0 ? &tm_dk : &tm_dv;
+      uint8_t* stage = smem + L::kK + (g * 4 + wq) * (HD / 64) * 4096;
+#pragma unroll 1
+      for (int rd = 0; rd < 2; ++rd) {
+#pragma unroll 1
+        for (int cb = 0; cb < HD / 64; ++cb) {
+          const int col = (rd * (HD / 64) + cb) * 32;
+          store_box(tacc + lane_off + col, stage + cb * 4096, m, h * HD + col,
+                    int32_t(kb) + wq * 32, lane);
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.error, HSTU_DEVERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ================================================================ key-tile order
+
+// One block: per key tile the number of query tiles that can see it (from the
+// tile to the end of the user owning its last row), then a counting sort by
+// descending count (longest processing time first).
+__global__ void key_order_kernel(const RowInfo* __restrict__ rows,
+                                 const int32_t* __restrict__ offsets, int32_t B, int64_t T,
+                                 int32_t nkt, int32_t* __restrict__ cost,
+                                 int32_t* __restrict__ order) {
+  constexpr int NB = 4096;
+  __shared__ int32_t hist[NB];
+  __shared__ int32_t s_max;
+  for (int c = threadIdx.x; c < NB; c += blockDim.x) hist[c] = 0;
+  if (threadIdx.x == 0) s_max = 0;
+  __syncthreads();
+  int32_t local_max = 0;
+  for (int32_t kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
+    const int64_t kb = int64_t(kt) * 128;
+    const int64_t r_last = kb + 127 < T ? kb + 127 : T - 1;
+    int32_t u = rows[r_last].user;
+    u = u < 0 ? 0 : (u >= B ? B - 1 : u);
+    int64_t ue = offsets[u + 1];
+    if (ue <= r_last) ue = r_last + 1;
+    if (ue > T) ue = T;
+    const int32_t c = int32_t((ue + 127) / 128) - kt;
+    cost[kt] = c;
+    local_max = c > local_max ? c : local_max;
+    atomicAdd(&hist[c < NB ? c : NB - 1], 1);
+  }
+  atomicMax(&s_max, local_max);
+  __syncthreads();
+  const int top = s_max < NB ? s_max : NB - 1;
+  if (threadIdx.x == 0) {
+    int32_t run = 0;
+    for (int c = top; c >= 0; --c) {
+      const int32_t n = hist[c];
+      hist[c] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  for (int32_t kt = threadIdx.x; kt < nkt; kt += blockDim.x) {
+    const int32_t c = cost[kt];
+    const int32_t slot = atomicAdd(&hist[c < NB ? c : NB - 1], 1);
+    order[slot] = kt;
+  }
+}
+
 // ==== host side: launch configuration (no device code below this line) ====
 
 template <int HD>
-cudaError_t launch_bwd_hd(const AttnBwdArgs& a, cudaStream_t st) {
-  using L = BwdLayout<HD>;
-  CUtensorMap tm, tm_do, tm_ts;
+cudaError_t launch_bwd_hd(const AttnBwdArgs& a, const BwdParams& p, cudaStream_t st) {
+  CUtensorMap tm, tm_do, tm_ts, tm_rows, tm_dq, tm_dk, tm_dv;
   if (!make_tmap_2d_bf16(&tm, a.uvqk, uint64_t(4 * a.d), uint64_t(a.T), uint64_t(4 * a.d) * 2,
                          64, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tm_do, a.dO, uint64_t(a.d), uint64_t(a.T), uint64_t(a.d) * 2, 64, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_1d_i64(&tm_ts, a.ts, uint64_t(a.T), 128)) return cudaErrorInvalidValue;
-  static std::atomic<uint64_t> smem_set{0};
-  const cudaError_t e = smem_opt_in(attn_bwd_tc_kernel<HD>, int(L::smem_bytes(kBwdMaxPos - 1)),
-                                    smem_set);
+  if (!make_tmap_1d_i64(&tm_rows, a.rows, uint64_t(a.T) * 2, 256)) return cudaErrorInvalidValue;
+  const uint64_t dd = uint64_t(a.d), tt = uint64_t(a.T);
+  if (!make_tmap_2d_f32_sw128(&tm_dq, a.dq, dd, tt, dd * 4, 32, 32) ||
+      !make_tmap_2d_f32_sw128(&tm_dk, a.dk, dd, tt, dd * 4, 32, 32) ||
+      !make_tmap_2d_f32_sw128(&tm_dv, a.dv, dd, tt, dd * 4, 32, 32))
+    return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> set_dq{0}, set_dkv{0};
+  cudaError_t e = smem_opt_in(attn_bwd_dq_kernel<HD>,
+                              int(DqLayout<HD>::smem_bytes(kBwdMaxPos - 1)), set_dq);
+  if (e == cudaSuccess)
+    e = smem_opt_in(attn_bwd_dkv_kernel<HD>, int(DkvLayout<HD>::kSmemBytes), set_dkv);
   if (e != cudaSuccess) return e;
-  AttnBwdParams p;
-  p.rows = a.rows;
-  p.offsets = a.offsets;
-  p.B = a.B;
-  p.ts = a.ts;
-  p.thresholds = a.thresholds;
-  p.rab_pos = a.rab_pos;
-  p.rab_time = a.rab_time;
-  p.counters = a.counters;
-  p.error = a.error;
-  p.dq = a.dq;
-  p.dk = a.dk;
-  p.dv = a.dv;
-  p.d_rab_pos = a.d_rab_pos;
-  p.d_rab_time = a.d_rab_time;
-  p.T = a.T;
-  p.d = a.d;
-  p.H = a.H;
-  p.num_key_tiles = int((a.T + 127) / 128);
-  p.pos_clamp = a.pos_clamp;
-  p.time_buckets = a.time_buckets;
-  p.n_norm_fixed = a.n_norm_fixed;
-  const int64_t grid = int64_t(p.num_key_tiles) * a.H;
-  attn_bwd_tc_kernel<HD><<<unsigned(grid), kBwdThreads, L::smem_bytes(a.pos_clamp), st>>>(
-      tm, tm_do, tm_ts, p);
+  const int64_t grid_q = int64_t(2) * p.num_pairs * a.H;
+  attn_bwd_dq_kernel<HD><<<unsigned(grid_q), kBwdThreads, DqLayout<HD>::smem_bytes(a.pos_clamp),
+                           st>>>(tm, tm_do, tm_ts, tm_dq, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t grid_k = int64_t(p.num_key_tiles) * a.H;
+  attn_bwd_dkv_kernel<HD><<<unsigned(grid_k), kBwdThreads, DkvLayout<HD>::kSmemBytes, st>>>(
+      tm, tm_do, tm_ts, tm_rows, tm_dk, tm_dv, p);
   return cudaGetLastError();
 }
 
@@ -485,9 +948,38 @@ cudaError_t launch_bwd_hd(const AttnBwdArgs& a, cudaStream_t st) {
 cudaError_t launch_attention_bwd_tc(const AttnBwdArgs& a, cudaStream_t st) {
   if (a.T <= 0 || a.B <= 0) return cudaSuccess;
   if (a.pos_clamp >= kBwdMaxPos || a.time_buckets > kBwdMaxBuckets) return cudaErrorInvalidValue;
-  if (a.hd == 128) return launch_bwd_hd<128>(a, st);
-  if (a.hd == 64) return launch_bwd_hd<64>(a, st);
-  return cudaErrorInvalidValue;
+  if (a.hd != 128 && a.hd != 64) return cudaErrorInvalidValue;
+  BwdParams p;
+  p.rows = a.rows;
+  p.order = a.order;
+  p.key_order = a.key_order;
+  p.offsets = a.offsets;
+  p.B = a.B;
+  p.ts = a.ts;
+  p.thresholds = a.thresholds;
+  p.time_lut = a.time_lut;
+  p.thr32 = a.thr32;
+  p.rab_pos = a.rab_pos;
+  p.rab_time = a.rab_time;
+  p.counters = a.counters;
+  p.error = a.error;
+  p.d_rab_pos = a.d_rab_pos;
+  p.d_rab_time = a.d_rab_time;
+  p.T = a.T;
+  p.d = a.d;
+  p.H = a.H;
+  p.num_pairs = int((a.T + 2 * kTile - 1) / (2 * kTile));
+  p.num_key_tiles = int((a.T + kTile - 1) / kTile);
+  p.pos_clamp = a.pos_clamp;
+  p.time_buckets = a.time_buckets;
+  p.n_norm_fixed = a.n_norm_fixed;
+  p.lut_exact = a.lut_exact;
+  p.wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimit;
+  key_order_kernel<<<1, 1024, 0, st>>>(a.rows, a.offsets, a.B, a.T, p.num_key_tiles, a.key_cost,
+                                       a.key_order);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return a.hd == 128 ? launch_bwd_hd<128>(a, p, st) : launch_bwd_hd<64>(a, p, st);
 }
 
 }  // namespace hstu

@@ -98,6 +98,7 @@ struct AttnParams {
   int pos_clamp, time_buckets;
   int n_norm_fixed;
   int lut_exact;
+  long long wait_limit;
   int32_t* dump_pidx;
   int32_t* dump_tidx;
   uint8_t* dump_vis;
@@ -216,8 +217,13 @@ __device__ __forceinline__ float score_one(float acc, int jr, int64_t tk, Row& R
     // masked keys may hold any gap (even -1, i.e. v = 0): keep v >= 1 so the
     // table index stays in [0, 127] for every input
     const uint32_t v = max(dd + 1u, 1u);
-    const int lz = __clz(int(v));
-    const int idx = (((31 - lz) << 2) | int((v << lz) >> 29 & 3u)) & 127;
+    // the bin index floor(log2 v) * 4 + the next two bits of v, read off the
+    // exponent and top mantissa bits of v converted with truncation (exact:
+    // truncation never carries into the exponent); the conversion runs beside
+    // the tanh instead of competing with it on the multi-function unit, as a
+    // leading-zero count would
+    const uint32_t fb = __float_as_uint(__uint2float_rz(v));
+    const int idx = int((fb >> 21) - 508u) & 127;
     const int4 ent = reinterpret_cast<const int4*>(s_lut)[idx];   // {thr, rt_lo, rt_hi, cand}
     const bool up = int(dd) >= ent.x;
     const float rt = __int_as_float(up ? ent.z : ent.y);
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int s = j % NSK;
         const uint32_t ph = (j / NSK) & 1;
-        if (!mbar_wait(&k_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&k_empty[s], ph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
@@ -458,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the tile's key timestamps (a deeper ring: the row groups classify ahead)
         const int st = j % NST;
         const uint32_t tph = (j / NST) & 1;
-        if (!mbar_wait(&t_empty[st], tph ^ 1)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&t_empty[st], tph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&t_full[st], 128 * 8);
         tma_load_1d(s_kts + st * 128, &tm_ts, &t_full[st], key_tile(j) * 128);
         t_issued[st] = true;
@@ -479,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int s = j % NSV;
         const uint32_t ph = (j / NSV) & 1;
-        if (!mbar_wait(&v_empty[s], ph ^ 1)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&v_empty[s], ph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
 #pragma unroll
         for (int b = 0; b < HD / 64; ++b)
@@ -500,13 +506,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && q < nq) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, HD, false, true);
-      bool ok = mbar_wait(q_full, 0);
+      bool ok = mbar_wait(q_full, 0, p.wait_limit);
       tc_fence_after();
       const uint32_t sQ = smem_u32(smem + L::kQ + q * L::kTileBytes);
       // S_q = Q_q K_j^T; the K stage is released once every issuer's product has read it
       auto issue_qk = [&](int j) -> bool {
         const int s = j % NSK;
-        if (!mbar_wait(&k_full[s], (j / NSK) & 1)) return false;
+        if (!mbar_wait(&k_full[s], (j / NSK) & 1, p.wait_limit)) return false;
         tc_fence_after();
         const uint32_t sK = smem_u32(smem + L::kK + s * L::kTileBytes);
 #pragma unroll
@@ -523,8 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool o_done = false;
       for (int j = 0; ok && j < n_kt; ++j) {
         const int s = j % NSV;
-        if (!mbar_wait(&v_full[s], (j / NSV) & 1)) { ok = false; break; }
-        if (!mbar_wait(&p_full[q], j & 1)) { ok = false; break; }
+        if (!mbar_wait(&v_full[s], (j / NSV) & 1, p.wait_limit)) { ok = false; break; }
+        if (!mbar_wait(&p_full[q], j & 1, p.wait_limit)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sV = smem_u32(smem + L::kV + s * L::kTileBytes);
 #pragma unroll
@@ -628,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t* kts = s_kts + st * 128;
       // The key timestamps of tile j come through their own ring, loaded well
       // ahead of the scores: classify the rows first, off the critical path.
-      bool ok = aborted ? false : mbar_wait(&t_full[st], (j / NST) & 1);
+      bool ok = aborted ? false : mbar_wait(&t_full[st], (j / NST) & 1, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         aborted = true;
@@ -698,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       rec.kb = kb;
       rec.on = RECORD && h == 0 && valid;
 
-      ok = mbar_wait(&s_full[q], j & 1);
+      ok = mbar_wait(&s_full[q], j & 1, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         aborted = true;
@@ -740,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // columns, per warp) -> TMA stores, which clip the rows past T.  Once o_full[q]
     // fired, every MMA of this query tile is done, so Q_q's tile is free to stage in.
     if (q < nq) {
-      bool ok = aborted ? false : mbar_wait(&o_full[q], 0);
+      bool ok = aborted ? false : mbar_wait(&o_full[q], 0, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
@@ -812,6 +818,7 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
   p.time_lut = a.time_lut;
   p.thr32 = a.thr32;
   p.lut_exact = a.lut_exact;
+  p.wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimit;
   p.rab_pos = a.rab_pos;
   p.rab_time = a.rab_time;
   p.counters = a.counters;

@@ -41,6 +41,7 @@ struct GemmParams {
   const void* residual;
   int io_fp32;
   int out_bf16;         // fp32 out: also store bf16(out) through tma_out2
+  long long wait_limit; // bound of the pipeline waits (the drains keep the default)
   int32_t* error;
 };
 
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int64_t mt = t / n_tiles;
         const int nt = int(t % n_tiles);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
           uint8_t* sa = smem + stage * L::kStageBytes;
           tma_load_2d(sa, &tma_a, &full[stage], kb * kBK, int32_t(mt * 128));
@@ -145,11 +146,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool any = false;
       for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+          if (!mbar_wait(&full[stage], phase, p.wait_limit)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * L::kStageBytes);
           const uint32_t b_addr = a_addr + L::kABytes;
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
-      if (!mbar_wait(&acc_full[acc], acc_phase)) { *abort_flag = 1; break; }
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.wait_limit)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int64_t mt = t / n_tiles;
       const int nt = int(t % n_tiles);
@@ -330,6 +331,7 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   p.residual = a.residual;
   p.io_fp32 = a.io_fp32;
   p.out_bf16 = copy ? 1 : 0;
+  p.wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimit;
   p.error = error;
   const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
   const int grid = int(tiles < num_sms ? tiles : num_sms);

@@ -215,6 +215,8 @@ hstu_status hstu_create(const hstu_config* cfg, int32_t device, hstu_handle** ou
   if (e == cudaSuccess) e = hstu::alloc(&ws.rows, T * sizeof(hstu::RowInfo));
   if (e == cudaSuccess) e = hstu::alloc(&ws.qtile_order, nqt * 4);
   if (e == cudaSuccess) e = hstu::alloc(&ws.qtile_cost, nqt * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.ktile_order, nqt * 4);
+  if (e == cudaSuccess) e = hstu::alloc(&ws.ktile_cost, nqt * 4);
   if (e == cudaSuccess) e = hstu::alloc(&ws.counters, 16);
   if (e == cudaSuccess) e = hstu::alloc(&ws.error, 16);
   if (e == cudaSuccess) e = hstu::alloc(&ws.thresholds, 256 * 8);
@@ -241,7 +243,8 @@ hstu_status hstu_destroy(hstu_handle* h) {
   cudaDeviceSynchronize();
   Workspace& ws = h->ws;
   void* ptrs[] = {ws.xb, ws.uvqk, ws.av, ws.g, ws.rows, ws.qtile_order, ws.qtile_cost,
-                  ws.counters, ws.error, ws.thresholds, ws.time_lut, ws.thr32};
+                  ws.ktile_order, ws.ktile_cost, ws.counters, ws.error, ws.thresholds,
+                  ws.time_lut, ws.thr32};
   for (void* p : ptrs)
     if (p != nullptr) cudaFree(p);
   hstu::BwdWorkspace& bw = h->bwd;
@@ -369,6 +372,8 @@ hstu_status run_layer(hstu_handle* h, const void* x, const LayerRows& R,
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
   a.num_pairs = R.num_pairs;
+  a.wait_limit = h->wait_limit;
+  a.q_row0 = R.q0;
   if (f32) {
     {
       Timed tm(h, kF1, st);
@@ -412,6 +417,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, const LayerRows& R,
   g1.residual = nullptr;
   g1.io_fp32 = 0;
   g1.out_bf16 = nullptr;
+  g1.wait_limit = h->wait_limit;
   if (e == cudaSuccess) {
     Timed tm(h, kF1, st);
     e = hstu::launch_gemm_tc(g1, h->num_sms, st, ws.error);
@@ -436,6 +442,7 @@ hstu_status run_layer(hstu_handle* h, const void* x, const LayerRows& R,
   g2.residual = x;
   g2.io_fp32 = io32 ? 1 : 0;
   g2.out_bf16 = (io32 && make_xb) ? ws.xb : nullptr;
+  g2.wait_limit = h->wait_limit;
   if (e == cudaSuccess) {
     Timed tm(h, kF2, st);
     e = hstu::launch_gemm_tc(g2, h->num_sms, st, ws.error);
@@ -568,6 +575,12 @@ hstu_status hstu_debug_attention_buckets(hstu_handle* h, int64_t T, const int32_
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   cudaFree(zeros);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status hstu_set_wait_limit(hstu_handle* h, int64_t cycles) {
+  if (h == nullptr || cycles < 0) return HSTU_ERR_INVALID_ARG;
+  h->wait_limit = cycles;
+  return HSTU_OK;
 }
 
 hstu_status hstu_set_kernel_timing(hstu_handle* h, int32_t enabled) {
@@ -1121,6 +1134,7 @@ extern "C" hstu_status hstu_attention_forward(hstu_handle* h, const void* uvqk, 
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
   a.num_pairs = int((T + 2 * hstu::kTile - 1) / (2 * hstu::kTile));
+  a.wait_limit = h->wait_limit;
   {
     Timed tm(h, kAttention, st);
     e = c.compute_dtype == HSTU_DTYPE_FP32 ? hstu::launch_attention_f32(a, st)
@@ -1131,36 +1145,29 @@ extern "C" hstu_status hstu_attention_forward(hstu_handle* h, const void* uvqk, 
 
 // ---------------------------------------------------------------------------
 // Backward of the attention step
-extern "C" hstu_status hstu_attention_backward(
-    hstu_handle* h, const void* uvqk, const void* d_out, int64_t T, const int32_t* offsets,
-    int32_t B, const int64_t* ts, hstu_mask_mode mode, const int32_t* ncand, const float* rab_pos,
-    const float* rab_time, float* dq, float* dk, float* dv, float* d_rab_pos, float* d_rab_time,
-    void* stream) {
-  hstu_status s = check_common(h, uvqk, T, offsets, B, ts, mode, ncand, d_out);
-  if (s != HSTU_OK) return s;
-  if (h->cfg.compute_dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
-  if (T == 0) return HSTU_OK;
-  const void* ps[] = {rab_pos, rab_time, dq, dk, dv, d_rab_pos, d_rab_time};
-  for (const void* q : ps)
-    if (q == nullptr || !hstu::aligned16(q)) return HSTU_ERR_INVALID_ARG;
-  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+namespace {
+
+// The attention backward's arguments on the handle's schedule (launch_schedule
+// must have run on the same batch).
+hstu::AttnBwdArgs bwd_args(hstu_handle* h, const void* uvqk, const void* d_out, int64_t T,
+                           const int32_t* offsets, int32_t B, const int64_t* ts,
+                           const float* rab_pos, const float* rab_time, float* dq, float* dk,
+                           float* dv, float* d_rab_pos, float* d_rab_time) {
   const hstu_config& c = h->cfg;
-  const size_t d = size_t(c.d_model);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dq, 0, size_t(T) * d * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_pos, 0, size_t(c.pos_buckets) * 4, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, size_t(c.time_buckets) * 4, st);
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
   hstu::AttnBwdArgs a;
   memset(&a, 0, sizeof(a));
   a.uvqk = uvqk;
   a.dO = d_out;
   a.rows = h->ws.rows;
+  a.order = h->ws.qtile_order;
+  a.key_cost = h->ws.ktile_cost;
+  a.key_order = h->ws.ktile_order;
   a.offsets = offsets;
   a.B = B;
   a.ts = ts;
   a.thresholds = h->ws.thresholds;
+  a.time_lut = h->ws.time_lut;
+  a.thr32 = h->ws.thr32;
   a.rab_pos = rab_pos;
   a.rab_time = rab_time;
   a.counters = h->ws.counters;
@@ -1177,6 +1184,34 @@ extern "C" hstu_status hstu_attention_backward(
   a.pos_clamp = c.pos_clamp;
   a.time_buckets = c.time_buckets;
   a.n_norm_fixed = c.n_norm;
+  a.lut_exact = c.time_log_div > 0.2232 ? 1 : 0;
+  a.wait_limit = h->wait_limit;
+  return a;
+}
+
+}  // namespace
+
+extern "C" hstu_status hstu_attention_backward(
+    hstu_handle* h, const void* uvqk, const void* d_out, int64_t T, const int32_t* offsets,
+    int32_t B, const int64_t* ts, hstu_mask_mode mode, const int32_t* ncand, const float* rab_pos,
+    const float* rab_time, float* dq, float* dk, float* dv, float* d_rab_pos, float* d_rab_time,
+    void* stream) {
+  hstu_status s = check_common(h, uvqk, T, offsets, B, ts, mode, ncand, d_out);
+  if (s != HSTU_OK) return s;
+  if (h->cfg.compute_dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (T == 0) return HSTU_OK;
+  const void* ps[] = {rab_pos, rab_time, dq, dk, dv, d_rab_pos, d_rab_time};
+  for (const void* q : ps)
+    if (q == nullptr || !hstu::aligned16(q)) return HSTU_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu_config& c = h->cfg;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_pos, 0, size_t(c.pos_buckets) * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, size_t(c.time_buckets) * 4, st);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const hstu::AttnBwdArgs a = bwd_args(h, uvqk, d_out, T, offsets, B, ts, rab_pos, rab_time, dq,
+                                       dk, dv, d_rab_pos, d_rab_time);
   e = hstu::launch_attention_bwd_tc(a, st);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
@@ -1302,33 +1337,9 @@ extern "C" hstu_status hstu_layer_backward(
                                  b.dO, b.g, gr->ln_gamma, gr->ln_beta, h->num_sms, st);
   // the attention step (its schedule, then the backward kernel)
   if (e == cudaSuccess) e = hstu::launch_schedule(h, T, offsets, B, ts, mode, ncand, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(b.dq, 0, size_t(T) * d * 4, st);
   if (e == cudaSuccess) {
-    hstu::AttnBwdArgs a;
-    memset(&a, 0, sizeof(a));
-    a.uvqk = uvqk;
-    a.dO = b.dO;
-    a.rows = h->ws.rows;
-    a.offsets = offsets;
-    a.B = B;
-    a.ts = ts;
-    a.thresholds = h->ws.thresholds;
-    a.rab_pos = w->rab_pos;
-    a.rab_time = w->rab_time;
-    a.counters = h->ws.counters;
-    a.error = h->ws.error;
-    a.dq = b.dq;
-    a.dk = b.dk;
-    a.dv = b.dv;
-    a.d_rab_pos = gr->rab_pos;
-    a.d_rab_time = gr->rab_time;
-    a.T = T;
-    a.d = d;
-    a.H = c.num_heads;
-    a.hd = c.head_dim;
-    a.pos_clamp = c.pos_clamp;
-    a.time_buckets = c.time_buckets;
-    a.n_norm_fixed = c.n_norm;
+    const hstu::AttnBwdArgs a = bwd_args(h, uvqk, b.dO, T, offsets, B, ts, w->rab_pos,
+                                         w->rab_time, b.dq, b.dk, b.dv, gr->rab_pos, gr->rab_time);
     e = hstu::launch_attention_bwd_tc(a, st);
   }
   // SiLU: H1 recomputed, dH1 = dZ (.) SiLU'(H1), b1 gradient

@@ -77,6 +77,8 @@ struct Workspace {
   RowInfo* rows = nullptr;     // [T]
   int32_t* qtile_order = nullptr;  // [ceil(T / 256)] q-tile pairs by descending cost
   int32_t* qtile_cost = nullptr;   // [ceil(T / 256)]
+  int32_t* ktile_order = nullptr;  // [ceil(T / 128)] key tiles of the backward, longest first
+  int32_t* ktile_cost = nullptr;   // [ceil(T / 128)]
   int32_t* counters = nullptr;     // [4]: n_norm, max cost, scratch
   int32_t* error = nullptr;        // device error word
   int64_t* thresholds = nullptr;   // [time_buckets] time-bucket thresholds
@@ -132,6 +134,7 @@ struct hstu_handle_s {
   int num_sms = 148;
   hstu::Workspace ws;
   int64_t last_T = 0;
+  int64_t wait_limit = 0;     // pipeline wait bound of the tensor-core kernels (0: default)
   int64_t thresholds_host[256];
   uint8_t time_lut_host[128];
   int32_t thr32_host[257];
@@ -203,6 +206,8 @@ struct GemmArgs {
   // kBiasResidual with fp32 out only: when set, bf16(out) is written here too
   // (the next layer's f1 operand), rounded to nearest even
   void* out_bf16;
+  // bound of the pipeline waits in SM cycles (0: the default, about a second)
+  int64_t wait_limit = 0;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error);
 
@@ -226,6 +231,8 @@ struct AttnArgs {
   int n_norm_fixed;          // > 0: use it; else counters[0]
   int num_pairs;             // ceil(T / 256)
   int lut_exact;             // time_log_div > ln 1.25: the candidate-bucket table is exact
+  int64_t wait_limit;        // bound of the pipeline waits in SM cycles (0: the default)
+  int64_t q_row0;            // first row of the listed pairs (rows [q_row0, T) are written)
   // recording variant
   int32_t* dump_pidx;
   int32_t* dump_tidx;
@@ -237,16 +244,21 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t st, bool record)
 struct AttnBwdArgs {
   const void* uvqk;          // [T, 4d] bf16 (the forward's U | V | Q | K)
   const void* dO;            // [T, d] bf16: gradient of the attention output O
-  const RowInfo* rows;       // the forward's row facts
+  const RowInfo* rows;       // the forward's row facts (the schedule)
+  const int32_t* order;      // query-tile pairs, longest first (the schedule)
+  int32_t* key_cost;         // [ceil(T / 128)] scratch: query tiles per key tile
+  int32_t* key_order;        // [ceil(T / 128)] scratch: key tiles, longest first
   const int32_t* offsets;    // [B + 1]
   int32_t B;
   const int64_t* ts;
   const int64_t* thresholds; // [time_buckets]
+  const uint8_t* time_lut;   // [128]
+  const int32_t* thr32;      // [257]
   const float* rab_pos;
   const float* rab_time;
   const int32_t* counters;   // [0] = n_norm when not fixed
   int32_t* error;
-  float* dq;                 // [T, d] fp32, zeroed by the caller (accumulated)
+  float* dq;                 // [T, d] fp32 (written)
   float* dk;                 // [T, d] fp32 (written)
   float* dv;                 // [T, d] fp32 (written)
   float* d_rab_pos;          // [pos_buckets] fp32, zeroed by the caller (accumulated)
@@ -254,6 +266,8 @@ struct AttnBwdArgs {
   int64_t T;
   int d, H, hd;
   int pos_clamp, time_buckets, n_norm_fixed;
+  int lut_exact;             // time_log_div > ln 1.25: the bin table of the buckets is exact
+  int64_t wait_limit;        // bound of the pipeline waits in SM cycles (0: the default)
 };
 cudaError_t launch_attention_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
 

@@ -49,14 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `parity` to complete, for at most ~2^31 SM cycles
-// (about a second).  Returns false on timeout; the caller records the error
-// and winds down instead of spinning forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// The default bound of a wait: 2^31 SM cycles, about a second.
+constexpr long long kWaitLimit = 1LL << 31;
+
+// Waits for the phase of `parity` to complete, for at most `limit` SM cycles.
+// Returns false on timeout; the caller records the error and winds down
+// instead of spinning forever.  Waits that drain a CTA's own copies and MMAs
+// before it exits always take the default bound.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit = kWaitLimit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > (1LL << 31)) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }
@@ -98,6 +103,18 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                    reinterpret_cast<uint64_t>(m)),
                "r"(smem_u32(smem_src)), "r"(x), "r"(y)
                : "memory");
+}
+
+// 2-D tiled bulk tensor reduction shared -> global: adds the fp32 box element
+// by element into the tensor (bulk-group completion).  Same coordinate rules
+// as tma_store_2d.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* smem_src,
+                                                  int32_t x, int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], "
+      "[%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+      : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit_group() {

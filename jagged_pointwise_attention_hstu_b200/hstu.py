@@ -123,6 +123,7 @@ def load() -> ctypes.CDLL:
                                         c_void_p, c_int32, c_void_p,
                                         POINTER(hstu_layer_weights), c_int, c_void_p, c_void_p,
                                         POINTER(hstu_layer_grads), c_void_p]),
+        "hstu_set_wait_limit": (c_int, [H, c_int64]),
         "hstu_set_kernel_timing": (c_int, [H, c_int32]),
         "hstu_get_kernel_timing": (c_int, [H, POINTER(c_double), POINTER(c_int64)]),
     }
@@ -335,6 +336,10 @@ def hstu_layer_backward(handle, values, uvqk, av, d_out, total_tokens: int, seq_
                                       _ptr(num_candidates), _ptr(d_values), ctypes.byref(g),
                                       _stream_ptr(stream)),
            "hstu_layer_backward")
+
+
+def hstu_set_wait_limit(handle, cycles: int) -> None:
+    _check(load().hstu_set_wait_limit(handle, cycles), "hstu_set_wait_limit")
 
 
 KERNEL_KINDS = ("schedule", "cast", "f1", "attention", "ln_gate", "f2", "block")

@@ -20,7 +20,7 @@ int main(void) {
       (any_fn)hstu_stochastic_length, (any_fn)hstu_copy_intermediate,
       (any_fn)hstu_debug_attention_buckets, (any_fn)hstu_debug_umma_tile,
       (any_fn)hstu_attention_backward, (any_fn)hstu_layer_backward,
-      (any_fn)hstu_attention_forward};
+      (any_fn)hstu_attention_forward, (any_fn)hstu_set_wait_limit};
   size_t i, n = sizeof(entry_points) / sizeof(entry_points[0]);
   for (i = 0; i < n; ++i)
     if (entry_points[i] == NULL) return 2;

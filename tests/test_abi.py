@@ -101,6 +101,7 @@ def test_null_arguments_are_rejected(lib):
                                        None) == hstu.HSTU_ERR_INVALID_ARG
     assert lib.hstu_attention_forward(None, None, 0, None, 0, None, 0, None, None, None, None,
                                       None) == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_set_wait_limit(None, 0) == hstu.HSTU_ERR_INVALID_ARG
 
 
 def test_stochastic_length_host_checks(lib):

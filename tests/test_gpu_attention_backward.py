@@ -80,6 +80,9 @@ def _rms(x):
     ("mfalcon", [300, 140, 260], [100, 140, 129], 4, 512),
     # n_norm = the longest user of the batch, found on the device by the schedule
     ("causal", [40, 300, 0, 129], None, 2, 0),
+    # a long user: most half tiles take the constant-bias path (every pair visible,
+    # clamped position, one time bucket per row)
+    ("causal", [1100, 37], None, 2, 1200),
 ])
 def test_attention_backward_teacher_forced(mask, lengths, ncand, H, n_norm):
     d = 256
