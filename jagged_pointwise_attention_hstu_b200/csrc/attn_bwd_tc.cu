@@ -76,8 +76,16 @@ struct BwdParams {
   int64_t T;
   int d, H, num_pairs, num_key_tiles;
   int pos_clamp, time_buckets, n_norm_fixed, lut_exact;
+  int rp_smem;                 // the padded rab_pos copy is in shared memory
   long long wait_limit;
 };
+
+// The shared copy of rab_pos is padded on both sides with its end values, so a
+// relative position in [-kPosPad, clamp + kPosPad] reads its clamped entry.
+constexpr int kPosPad = 130;
+__host__ __device__ constexpr uint32_t rp_bytes(int clamp) {
+  return ((uint32_t(clamp + 1 + 2 * kPosPad) * 4 + 15) / 16) * 16;
+}
 
 // ---------------------------------------------------------------- shared helpers
 
@@ -92,26 +100,25 @@ __device__ __forceinline__ int bucket_search(const int64_t* thr, int nb, int64_t
   return lo;
 }
 
-// Exact time bucket of a gap and its bias.  Gaps below 2^31 - 1 with a divisor
-// whose bins are narrower than a bucket: v = dt + 1 falls in the bin
-// floor(log2 v) * 4 + (next two bits), read off v converted with truncation;
-// the bin's entry holds the next bucket's threshold and both candidate biases.
-// Anything else: a binary search of the thresholds.
-__device__ __forceinline__ int time_bucket(int64_t dt, bool lut, const int4* s_any,
-                                           const int64_t* s_thr, const float* s_rt, int nb,
-                                           float& rt) {
-  if (dt < 0) dt = 0;
-  if (lut && dt < int64_t(0x7FFFFFFE)) {
-    const uint32_t v = uint32_t(dt) + 1u;
-    const uint32_t fb = __float_as_uint(__uint2float_rz(v));
-    const int4 e = s_any[int((fb >> 21) - 508u) & 127];
-    const bool up = int(dt) >= e.x;
-    rt = __int_as_float(up ? e.z : e.y);
-    return e.w + (up ? 1 : 0);
+// Time bias and bucket of a 32-bit gap through the bin table (the table is
+// exact for the divisor and the gap is below 2^31 - 1); a masked pair may hold
+// any 32-bit pattern, and its index stays inside the table.
+__device__ __forceinline__ float time_bias_lut(uint32_t dd, const int4* s_any, int& tb) {
+  const uint32_t v = max(dd + 1u, 1u);
+  const uint32_t fb = __float_as_uint(__uint2float_rz(v));
+  const int4 e = s_any[int((fb >> 21) - 508u) & 127];
+  const bool up = int(dd) >= e.x;
+  tb = e.w + (up ? 1 : 0);
+  return __int_as_float(up ? e.z : e.y);
+}
+
+// The padded rab_pos copy, written by the 256 row-group threads.
+__device__ __forceinline__ void load_rp(const BwdParams& p, int t, float* s_rp) {
+  const int n = p.pos_clamp + 1 + 2 * kPosPad;
+  for (int k = t; k < n; k += 256) {
+    const int q = k - kPosPad;
+    s_rp[k] = __ldg(p.rab_pos + (q < 0 ? 0 : (q > p.pos_clamp ? p.pos_clamp : q)));
   }
-  const int b = bucket_search(s_thr, nb, dt);
-  rt = s_rt[b];
-  return b;
 }
 
 // The per-CTA tables, written by the 256 row-group threads (t = 0..255).
@@ -194,15 +201,18 @@ struct DqLayout {
   static constexpr uint32_t kGtime = kRt + 1024;            // float [256]
   static constexpr uint32_t kAny = kGtime + 1024;           // int4 [128]
   static constexpr uint32_t kBars = kAny + 2048;
-  static constexpr uint32_t kGpos = kBars + 256;            // float [clamp + 1]
-  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
-    return kGpos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16 + 1024;
+  static constexpr uint32_t kGpos = kBars + 256;            // float [clamp + 1], then the rab_pos copy
+  static __host__ __device__ constexpr uint32_t rp_offset(int clamp) {
+    return kGpos + ((uint32_t(clamp + 1) * 4 + 15) / 16) * 16;
+  }
+  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp, bool rp) {
+    return rp_offset(clamp) + (rp ? rp_bytes(clamp) : 0) + 1024;
   }
   static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kTile % 1024 == 0, "tile alignment");
   static_assert(kKts % 128 == 0 && kBars % 8 == 0 && kAny % 16 == 0, "alignment");
   // dQ is staged in the Q and dO tiles: 8 warps x HD / 64 boxes of 4 KB
   static_assert(8 * (HD / 64) * 4096 == 2 * kTile, "dQ staging");
-  static_assert(smem_bytes(kBwdMaxPos - 1) <= 227 * 1024, "shared memory budget");
+  static_assert(smem_bytes(kBwdMaxPos - 1, false) <= 227 * 1024, "shared memory budget");
 };
 
 template <int HD>
@@ -235,6 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* s_gtime = reinterpret_cast<float*>(smem + L::kGtime);
   int4* s_any = reinterpret_cast<int4*>(smem + L::kAny);
   float* s_gpos = reinterpret_cast<float*>(smem + L::kGpos);
+  float* s_rp = reinterpret_cast<float*>(smem + L::rp_offset(p.pos_clamp));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;      // [NS]
@@ -272,6 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp >= 4) {
     const int t = threadIdx.x - 128;
     load_tables(p, t, s_thr, s_rt, s_any);
+    if (p.rp_smem) load_rp(p, t, s_rp);
     s_gtime[t] = 0.0f;
     for (int k = t; k <= clamp; k += 256) s_gpos[k] = 0.0f;
   }
@@ -366,23 +378,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int wq = warp & 3;                 // tensor-memory lane quarter
     const int row = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const int64_t i = r0 + row;
+    const int i = int(r0) + row;             // token indices fit in int32 (T <= 2^30)
     const bool valid = i < p.T;
-    int lo = 0, hi = 0, pos = 0;
-    int64_t ti = 0;
+    int lo = i, hi = i, pos = i;
+    int64_t ti = 0, t_first = 0;
     if (valid) {
       const RowInfo ri = p.rows[i];
-      lo = (ri.lo < 0 || ri.lo > i) ? int(i) : ri.lo;
+      lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
       hi = ri.hi;
       pos = ri.pos;
       ti = p.ts[i];
+      t_first = p.ts[lo];
     }
+    // every visible key of the row lies in its user at or after ts[lo]: below
+    // 2^31 - 1 its gap fits the 32-bit bin-table path
+    const bool narrow_row = !valid || ti - t_first < int64_t(0x7FFFFFFE);
+    const uint32_t ti_lo = uint32_t(ti);
     const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
-    const bool lut = p.lut_exact != 0;
+    const bool narrow = p.lut_exact != 0 && __all_sync(0xffffffffu, narrow_row);
     const float rp_clamp = __ldg(p.rab_pos + clamp);
+    const bool rp_smem = p.rp_smem != 0;
+    // position buckets along the tile diagonals: every row of the warp valid and
+    // positioned at its own index offset (history rows of one user)
+    const int pos0 = __shfl_sync(0xffffffffu, pos, 0);
+    const bool diag = __all_sync(0xffffffffu, valid && pos - lane == pos0);
+    const bool col = !diag && __all_sync(0xffffffffu, valid && pos == pos0);
     named_bar_sync(1, 256);   // the tables
     bool aborted = false;
+    float acc_c = 0.0f;       // the clamped position bucket's sum, added once at the end
     for (int j = 0; j < n_kt; ++j) {
       const int s = j % NS;
       const int kb = key_tile(j) * 128;
@@ -415,28 +439,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_st8(tS + tcol + 8 * c, pk);
       } else if (fast) {
-        // every pair visible, clamped position, one time bucket per row
+        // every pair visible, clamped position, one time bucket per row; the
+        // tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
         const float hc = rp_clamp + s_rt[tb0];
         float acc = 0.0f;
+        uint32_t xs[16], xa[16], ys[16], ya[16];
+        tmem_ld16(tS + tcol, xs);
+        tmem_ld16(tdA + tcol, xa);
+        tmem_ld_wait();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pk[8];
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld16(tS + tcol + 16 * (c + 1), ys);
+          tmem_ld16(tdA + tcol + 16 * (c + 1), ya);
+          {
+            uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const Grad g0 = silu_grad(__uint_as_float(rs[e]) + hc, __uint_as_float(ra[e]), inv_nn);
-            const Grad g1 =
-                silu_grad(__uint_as_float(rs[e + 1]) + hc, __uint_as_float(ra[e + 1]), inv_nn);
-            acc += g0.ds + g1.ds;
-            pk[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            for (int e = 0; e < 16; e += 2) {
+              const Grad g0 = silu_grad(__uint_as_float(xs[e]) + hc, __uint_as_float(xa[e]), inv_nn);
+              const Grad g1 = silu_grad(__uint_as_float(xs[e + 1]) + hc, __uint_as_float(xa[e + 1]), inv_nn);
+              acc += g0.ds + g1.ds;
+              pk[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            }
+            tmem_st8(tS + tcol + 8 * c, pk);
           }
-          tmem_st8(tS + tcol + 8 * c, pk);
+          tmem_ld_wait();
+          if (c + 2 < 4) {
+            tmem_ld16(tS + tcol + 16 * (c + 2), xs);
+            tmem_ld16(tdA + tcol + 16 * (c + 2), xa);
+          }
+          {
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const Grad g0 = silu_grad(__uint_as_float(ys[e]) + hc, __uint_as_float(ya[e]), inv_nn);
+              const Grad g1 = silu_grad(__uint_as_float(ys[e + 1]) + hc, __uint_as_float(ya[e + 1]), inv_nn);
+              acc += g0.ds + g1.ds;
+              pk[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            }
+            tmem_st8(tS + tcol + 8 * (c + 1), pk);
+          }
+          tmem_ld_wait();
         }
-        // the position bucket is the clamped one for the whole warp
+        acc_c += acc;   // the position bucket is the clamped one for every pair here
         const float wsum = warp_sum(acc);
-        if (lane == 0 && wsum != 0.0f) atomicAdd(s_gpos + clamp, wsum);
         if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
           if (lane == 0 && wsum != 0.0f) atomicAdd(s_gtime + tb0, wsum);
         } else if (acc != 0.0f) {
@@ -444,50 +489,110 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       } else {
         // any visibility: the mask, the position bucket and the exact time bucket
-        // of every pair; bias gradients summed along runs of one bucket
+        // of every pair.  The time-bucket gradient is summed along runs of one
+        // bucket; the position-bucket gradient along the tile diagonals (rows at
+        // their own positions: lane l gathers the pairs of its diagonal from the
+        // other lanes) or along the columns (rows at one position: M-FALCON
+        // candidates), else per pair.
+        const int pos_rel = min(max(pos - kb, -1), clamp + 129);
         int run_b = -1;
-        float run_acc = 0.0f, acc_c = 0.0f;
+        float run_acc = 0.0f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t rs[16], ra[16], pk[8];
+          const int jr0 = 64 * g + 16 * c;
           tmem_ld16(tS + tcol + 16 * c, rs);
           tmem_ld16(tdA + tcol + 16 * c, ra);
           tmem_ld_wait();
           float dsv[16];
+          int tbv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int jr = 64 * g + 16 * c + e;
+            const int jr = jr0 + e;
             const int jj = kb + jr;
-            const bool vis = valid && jj < p.T && ((lo <= jj && jj < hi) || int64_t(jj) == i);
+            const bool vis = valid && jj < p.T && ((lo <= jj && jj < hi) || jj == i);
             float rt;
-            const int tb = time_bucket(ti - kts[jr], lut, s_any, s_thr, s_rt, nb, rt);
-            int dp = pos - jj;
-            dp = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-            const float sc = __uint_as_float(rs[e]) + __ldg(p.rab_pos + dp) + rt;
-            const Grad gr = silu_grad(sc, __uint_as_float(ra[e]), inv_nn);
-            const float ds = vis ? gr.ds : 0.0f;
-            dsv[e] = ds;
-            if (vis) {
-              if (dp == clamp) acc_c += ds;
-              else atomicAdd(s_gpos + dp, ds);
-              if (tb != run_b) {
-                if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
-                run_b = tb;
-                run_acc = 0.0f;
-              }
-              run_acc += ds;
+            int tb;
+            if (narrow) {
+              rt = time_bias_lut(ti_lo - uint32_t(kts[jr]), s_any, tb);
+            } else {
+              int64_t gap = ti - kts[jr];
+              tb = bucket_search(s_thr, nb, gap < 0 ? 0 : gap);
+              rt = s_rt[tb];
             }
+            float rp;
+            if (rp_smem) {
+              rp = s_rp[kPosPad + pos_rel - jr];
+            } else {
+              int dp = pos - jj;
+              rp = __ldg(p.rab_pos + (dp < 0 ? 0 : (dp > clamp ? clamp : dp)));
+            }
+            const Grad gr = silu_grad(__uint_as_float(rs[e]) + rp + rt, __uint_as_float(ra[e]), inv_nn);
+            dsv[e] = vis ? gr.ds : 0.0f;
+            tbv[e] = vis ? tb : -1;
           }
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
           tmem_st8(tS + tcol + 8 * c, pk);
+          // time buckets: runs of one bucket along the row
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            if (tbv[e] < 0) continue;
+            if (tbv[e] != run_b) {
+              if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
+              run_b = tbv[e];
+              run_acc = 0.0f;
+            }
+            run_acc += dsv[e];
+          }
+          // position buckets
+          if (diag) {
+            // pair (lane l + e, column e) has position pos0 + l - (kb + jr0): lane l
+            // gathers them (and the wrapped ones, 32 positions lower)
+            float acc_a = 0.0f, acc_b = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float v = __shfl_sync(0xffffffffu, dsv[e], (lane + e) & 31);
+              if (lane + e < 32) acc_a += v; else acc_b += v;
+            }
+            const int da = pos0 + lane - (kb + jr0);
+            const int db = da - 32;
+            const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
+            const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
+            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) atomicAdd(s_gpos + ba, acc_a);
+            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) atomicAdd(s_gpos + bb, acc_b);
+          } else if (col) {
+            // one position per column: the column sums, lane e adds column e
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float v = dsv[e];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              if (lane == e && v != 0.0f) {
+                const int dp = pos0 - (kb + jr0 + e);
+                const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+                if (b == clamp) acc_c += v; else atomicAdd(s_gpos + b, v);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              if (dsv[e] == 0.0f) continue;
+              const int dp = pos - (kb + jr0 + e);
+              const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+              if (b == clamp) acc_c += dsv[e]; else atomicAdd(s_gpos + b, dsv[e]);
+            }
+          }
         }
         if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
-        if (acc_c != 0.0f) atomicAdd(s_gpos + clamp, acc_c);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
+    }
+    {
+      const float wsum = warp_sum(acc_c);
+      if (lane == 0 && wsum != 0.0f) atomicAdd(s_gpos + clamp, wsum);
     }
     if (aborted) *abort_flag = 1;
     // ---- dQ -> the (now free) Q and dO tiles -> TMA stores; the rows past T are clipped
@@ -543,12 +648,15 @@ struct DkvLayout {
   static constexpr uint32_t kRt = kThr + 2048;               // float [256]
   static constexpr uint32_t kAny = kRt + 1024;               // int4 [128]
   static constexpr uint32_t kBars = kAny + 2048;
-  static constexpr uint32_t kSmemBytes = kBars + 256 + 1024;
+  static constexpr uint32_t kRp = kBars + 256;               // the padded rab_pos copy
+  static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
+    return kRp + rp_bytes(clamp) + 1024;
+  }
   static_assert(kQ % 1024 == 0 && kDO % 1024 == 0 && kTile % 1024 == 0, "tile alignment");
   static_assert(kQf % 128 == 0 && kQts % 128 == 0 && kAny % 16 == 0, "alignment");
   // dK / dV are staged in the K and V tiles: 8 warps x HD / 64 boxes per pass, two passes
   static_assert(8 * (HD / 64) * 4096 == 2 * kTile, "dK / dV staging");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(smem_bytes(kBwdMaxPos - 1) <= 227 * 1024, "shared memory budget");
 };
 
 template <int HD>
@@ -581,6 +689,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
   float* s_rt = reinterpret_cast<float*>(smem + L::kRt);
   int4* s_any = reinterpret_cast<int4*>(smem + L::kAny);
+  float* s_rp = reinterpret_cast<float*>(smem + L::kRp);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* kv_full = bars;
   uint64_t* q_full = kv_full + 1;      // [NS] Q, dO and the query facts of a tile landed
@@ -615,7 +724,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  if (warp >= 4) load_tables(p, threadIdx.x - 128, s_thr, s_rt, s_any);
+  if (warp >= 4) {
+    load_tables(p, threadIdx.x - 128, s_thr, s_rt, s_any);
+    load_rp(p, threadIdx.x - 128, s_rp);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -714,19 +826,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const int64_t jk = kb + row;             // this thread's key
-    const bool valid = jk < p.T;
-    const int j = int(jk);
-    const int64_t tj = valid ? p.ts[jk] : 0;
+    const int j = int(kb) + row;             // this thread's key (T <= 2^30)
+    const bool valid = j < p.T;
+    int64_t tj = 0, t_last = 0;
+    if (valid) {
+      tj = p.ts[j];
+      // the queries that see key j lie in its user: their gaps are at most
+      // ts[end of user - 1] - t_j
+      int32_t u = p.rows[j].user;
+      u = u < 0 ? 0 : (u >= p.B ? p.B - 1 : u);
+      int64_t ue = p.offsets[u + 1];
+      ue = ue <= j ? j + 1 : (ue > p.T ? p.T : ue);
+      t_last = p.ts[ue - 1];
+    }
+    const bool narrow = p.lut_exact != 0 &&
+                        __all_sync(0xffffffffu, !valid || t_last - tj < int64_t(0x7FFFFFFE));
+    const uint32_t tj_lo = uint32_t(tj);
     const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
-    const bool lut = p.lut_exact != 0;
     const float rp_clamp = __ldg(p.rab_pos + clamp);
     named_bar_sync(1, 256);   // the tables
     bool aborted = false;
     for (int it = 0; it < nq; ++it) {
       const int s = it % NS;
-      const int64_t q0 = int64_t(kt + it) * 128;
+      const int q0 = (kt + it) * 128;
       bool ok = aborted ? false : mbar_wait(&q_full[s], (it / NS) & 1, p.wait_limit);
       ok = ok && mbar_wait(s_full, it & 1, p.wait_limit);
       ok = __all_sync(0xffffffffu, ok);
@@ -738,7 +861,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const RowInfo* qf = s_qf + s * 128;
       const int64_t* qts = s_qts + s * 128;
-      const int64_t i0 = q0 + 64 * g;   // first query of this group's half
+      const int i0 = q0 + 64 * g;   // first query of this group's half
       // ---- classify the key row for this half tile: the half's queries' facts,
       // reduced over the warp (each lane reads two)
       int mx_lo, mn_hi, mn_pos;
@@ -755,7 +878,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       const bool all_rows = i0 + 63 < p.T;
-      const bool zero = __all_sync(0xffffffffu, !valid || i0 + 63 < jk);
+      const bool zero = __all_sync(0xffffffffu, !valid || i0 + 63 < j);
       const bool full = valid && all_rows && mx_lo <= j && j < mn_hi;
       int tb0 = 0;
       bool same = false;
@@ -775,23 +898,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_st8(tdA + tcol + 8 * c, pk);
         }
       } else if (fast) {
+        // the tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
         const float hc = rp_clamp + s_rt[tb0];
+        uint32_t xs[16], xa[16], ys[16], ya[16];
+        tmem_ld16(tS + tcol, xs);
+        tmem_ld16(tdA + tcol, xa);
+        tmem_ld_wait();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pp[8], pd[8];
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld16(tS + tcol + 16 * (c + 1), ys);
+          tmem_ld16(tdA + tcol + 16 * (c + 1), ya);
+          {
+            uint32_t pp[8], pd[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const Grad g0 = silu_grad(__uint_as_float(rs[e]) + hc, __uint_as_float(ra[e]), inv_nn);
-            const Grad g1 =
-                silu_grad(__uint_as_float(rs[e + 1]) + hc, __uint_as_float(ra[e + 1]), inv_nn);
-            pp[e >> 1] = pack_bf16x2(g0.p, g1.p);
-            pd[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            for (int e = 0; e < 16; e += 2) {
+              const Grad g0 = silu_grad(__uint_as_float(xs[e]) + hc, __uint_as_float(xa[e]), inv_nn);
+              const Grad g1 = silu_grad(__uint_as_float(xs[e + 1]) + hc, __uint_as_float(xa[e + 1]), inv_nn);
+              pp[e >> 1] = pack_bf16x2(g0.p, g1.p);
+              pd[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            }
+            tmem_st8(tS + tcol + 8 * c, pp);
+            tmem_st8(tdA + tcol + 8 * c, pd);
           }
-          tmem_st8(tS + tcol + 8 * c, pp);
-          tmem_st8(tdA + tcol + 8 * c, pd);
+          tmem_ld_wait();
+          if (c + 2 < 4) {
+            tmem_ld16(tS + tcol + 16 * (c + 2), xs);
+            tmem_ld16(tdA + tcol + 16 * (c + 2), xa);
+          }
+          {
+            uint32_t pp[8], pd[8];
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const Grad g0 = silu_grad(__uint_as_float(ys[e]) + hc, __uint_as_float(ya[e]), inv_nn);
+              const Grad g1 = silu_grad(__uint_as_float(ys[e + 1]) + hc, __uint_as_float(ya[e + 1]), inv_nn);
+              pp[e >> 1] = pack_bf16x2(g0.p, g1.p);
+              pd[e >> 1] = pack_bf16x2(g0.ds, g1.ds);
+            }
+            tmem_st8(tS + tcol + 8 * (c + 1), pp);
+            tmem_st8(tdA + tcol + 8 * (c + 1), pd);
+          }
+          tmem_ld_wait();
         }
       } else {
 #pragma unroll 1
@@ -804,15 +950,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int ir = 64 * g + 16 * c + e;
-            const int64_t iq = q0 + ir;
+            const int iq = q0 + ir;
             const RowInfo f = qf[ir];
-            const bool vis = valid && iq < p.T && ((f.lo <= j && j < f.hi) || iq == jk);
+            const bool vis = valid && iq < p.T && ((f.lo <= j && j < f.hi) || iq == j);
             float rt;
-            time_bucket(qts[ir] - tj, lut, s_any, s_thr, s_rt, nb, rt);
-            int dp = f.pos - j;
-            dp = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-            const float sc = __uint_as_float(rs[e]) + __ldg(p.rab_pos + dp) + rt;
-            const Grad gr = silu_grad(sc, __uint_as_float(ra[e]), inv_nn);
+            if (narrow) {
+              int tb;
+              rt = time_bias_lut(uint32_t(qts[ir]) - tj_lo, s_any, tb);
+            } else {
+              const int64_t gap = qts[ir] - tj;
+              rt = s_rt[bucket_search(s_thr, nb, gap < 0 ? 0 : gap)];
+            }
+            // the position of pair (iq, j) relative to this key tile, clamped into
+            // the padded table
+            const int pr = min(max(f.pos - int(kb), -1), clamp + 129);
+            const float rp = s_rp[kPosPad + pr - row];
+            const Grad gr = silu_grad(__uint_as_float(rs[e]) + rp + rt, __uint_as_float(ra[e]), inv_nn);
             pv[e] = vis ? gr.p : 0.0f;
             dv[e] = vis ? gr.ds : 0.0f;
           }
@@ -927,18 +1080,23 @@ cudaError_t launch_bwd_hd(const AttnBwdArgs& a, const BwdParams& p, cudaStream_t
       !make_tmap_2d_f32_sw128(&tm_dv, a.dv, dd, tt, dd * 4, 32, 32))
     return cudaErrorInvalidValue;
   static std::atomic<uint64_t> set_dq{0}, set_dkv{0};
-  cudaError_t e = smem_opt_in(attn_bwd_dq_kernel<HD>,
-                              int(DqLayout<HD>::smem_bytes(kBwdMaxPos - 1)), set_dq);
+  cudaError_t e = smem_opt_in(attn_bwd_dq_kernel<HD>, 227 * 1024, set_dq);
   if (e == cudaSuccess)
-    e = smem_opt_in(attn_bwd_dkv_kernel<HD>, int(DkvLayout<HD>::kSmemBytes), set_dkv);
+    e = smem_opt_in(attn_bwd_dkv_kernel<HD>, int(DkvLayout<HD>::smem_bytes(kBwdMaxPos - 1)),
+                    set_dkv);
   if (e != cudaSuccess) return e;
+  // the dq kernel keeps the padded rab_pos copy in shared memory when it fits
+  BwdParams pq = p;
+  pq.rp_smem = DqLayout<HD>::smem_bytes(a.pos_clamp, true) <= 227 * 1024 ? 1 : 0;
   const int64_t grid_q = int64_t(2) * p.num_pairs * a.H;
-  attn_bwd_dq_kernel<HD><<<unsigned(grid_q), kBwdThreads, DqLayout<HD>::smem_bytes(a.pos_clamp),
-                           st>>>(tm, tm_do, tm_ts, tm_dq, p);
+  attn_bwd_dq_kernel<HD><<<unsigned(grid_q), kBwdThreads,
+                           DqLayout<HD>::smem_bytes(a.pos_clamp, pq.rp_smem != 0), st>>>(
+      tm, tm_do, tm_ts, tm_dq, pq);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t grid_k = int64_t(p.num_key_tiles) * a.H;
-  attn_bwd_dkv_kernel<HD><<<unsigned(grid_k), kBwdThreads, DkvLayout<HD>::kSmemBytes, st>>>(
+  attn_bwd_dkv_kernel<HD><<<unsigned(grid_k), kBwdThreads, DkvLayout<HD>::smem_bytes(a.pos_clamp),
+                            st>>>(
       tm, tm_do, tm_ts, tm_rows, tm_dk, tm_dv, p);
   return cudaGetLastError();
 }
@@ -974,6 +1132,7 @@ cudaError_t launch_attention_bwd_tc(const AttnBwdArgs& a, cudaStream_t st) {
   p.time_buckets = a.time_buckets;
   p.n_norm_fixed = a.n_norm_fixed;
   p.lut_exact = a.lut_exact;
+  p.rp_smem = 1;
   p.wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimit;
   key_order_kernel<<<1, 1024, 0, st>>>(a.rows, a.offsets, a.B, a.T, p.num_key_tiles, a.key_cost,
                                        a.key_order);
