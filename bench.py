@@ -113,6 +113,10 @@ def parse():
                          "16-user lognormal workload")
     ap.add_argument("--attn-bwd", action="store_true",
                     help="time the attention backward on one layer of the workload")
+    ap.add_argument("--cpu-plan", action="store_true",
+                    help="time the fp64 oracle on the host: configs 0, 1, 2, 4 whole (one "
+                         "layer), config 3 one full layer over all users (x layers: a labelled "
+                         "extrapolation); one JSON line per config")
     ap.add_argument("--train", action="store_true",
                     help="forward and backward of the stack per step (layer-tokens/s)")
     ap.add_argument("--layers", type=int, default=None,
@@ -213,12 +217,25 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(w, prefix, timed_layers=1):
-    """Times the fp64 oracle on one layer over user 0's causal prefix.
+REFERENCE_MAX_LEN = 8192
+
+
+def reference_sample_text(w):
+    if w.mask != "causal":
+        return f"1 layer over user 0 (history and candidates, {w.mask} mask), fp64 numpy oracle"
+    return (f"1 layer over user 0 (its first {REFERENCE_MAX_LEN} tokens at most, "
+            f"{w.mask} mask), fp64 numpy oracle")
+
+
+def oracle_sample(w, prefix=REFERENCE_MAX_LEN, timed_layers=1, num_users=1):
+    """Times the fp64 oracle on one layer over the first `num_users` users of the
+    workload's batch, each cut to its first `prefix` tokens (None: whole).
 
     Returns (seconds, layer-tokens processed)."""
     import oracle
-    batch = wl.make_batch(w, num_layers=1, num_users=1, max_len=prefix)
+    if w.mask != "causal":
+        prefix = None   # an M-FALCON user is taken whole (history and candidates)
+    batch = wl.make_batch(w, num_layers=1, num_users=num_users, max_len=prefix)
     lp = batch.layers[0]
     p = {k: np.asarray(getattr(lp, k), np.float32).astype(np.float64)
          for k in ("b1", "b2", "rab_pos", "rab_time", "ln_gamma", "ln_beta")}
@@ -273,15 +290,11 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = wl.WORKLOADS[args.workload]
-    prefix = 4096 if w.mask == "causal" else None
-    if prefix is None:
-        print(json.dumps({"impl": "reference", "unavailable": "reference sample defined for causal workloads"}))
-        return 0
     for _ in range(args.warmup):
-        oracle_sample(w, prefix)
+        oracle_sample(w)
     secs, units = 0.0, 0
     for _ in range(args.steps):
-        s, u = oracle_sample(w, prefix)
+        s, u = oracle_sample(w)
         secs += s
         units += u
     value = units / secs
@@ -292,9 +305,9 @@ def run_reference(args):
         "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "sample": f"1 layer over user 0's first {prefix} tokens per step"},
+        "config": {"workload": w.name, "sample": reference_sample_text(w) + " per step"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"1 layer x 1 user x {prefix}-token causal prefix per step"},
+                         "sample": reference_sample_text(w) + " per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -749,11 +762,30 @@ def launch_check(args):
     return spawn_ranks(args.gpus, os.path.abspath(__file__), sys.argv[1:])
 
 
+def run_cpu_plan(args):
+    """The oracle on the host cores, one JSON line per configuration: every user
+    of the batch through one layer (the stack's other layers are the same work
+    again, so config 3's 24 layers are extrapolated, and labelled so)."""
+    cores = blas_threads()
+    for idx in range(len(wl.WORKLOADS)):
+        w = wl.WORKLOADS[idx]
+        secs, units = oracle_sample(w, prefix=None, num_users=w.num_users)
+        line = {"impl": "oracle", "workload": w.name, "tokens": units, "layers_timed": 1,
+                "seconds": secs, "tokens_per_s": units / secs, "cores": cores}
+        if w.num_layers > 1:
+            line["stack_seconds_extrapolated"] = secs * w.num_layers
+            line["extrapolation"] = f"one layer timed, x {w.num_layers} layers"
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     rc = launch_check(args)
     if rc is not None:
         return rc
+    if args.cpu_plan:
+        return run_cpu_plan(args)
     if args.attn_bwd:
         return run_attn_bwd(args)
     if args.train:
@@ -945,13 +977,10 @@ def main():
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        prefix = 8192 if w.mask == "causal" else None
-        if prefix is not None:
-            secs, units = oracle_sample(w, min(prefix, int(batch.lengths[0])))
-            cpu_baseline = {"value": units / secs, "unit": "tokens/s", "cores": blas_threads(),
-                            "kind": "oracle",
-                            "sample": f"1 layer x user 0 ({min(prefix, int(batch.lengths[0]))} "
-                                      f"tokens), fp64 numpy, {secs:.1f} s"}
+        secs, units = oracle_sample(w)
+        cpu_baseline = {"value": units / secs, "unit": "tokens/s", "cores": blas_threads(),
+                        "kind": "oracle",
+                        "sample": reference_sample_text(w) + f", {units} tokens in {secs:.1f} s"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
