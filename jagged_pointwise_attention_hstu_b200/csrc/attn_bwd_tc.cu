@@ -424,13 +424,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // ---- classify the row for this half tile
       const bool zero = __all_sync(0xffffffffu, !valid || i < j0);
       const bool full = valid && lo <= j0 && j0 + 63 < hi;
-      int tb0 = 0;
+      int tb0 = 0, tb1 = 0;
       bool same = false;
       if (full) {
         tb0 = bucket_search(s_thr, nb, ti - kts[64 * g]);
-        same = tb0 == bucket_search(s_thr, nb, ti - kts[64 * g + 63]);
+        tb1 = bucket_search(s_thr, nb, ti - kts[64 * g + 63]);
+        same = tb0 == tb1;
       }
       const bool fast = __all_sync(0xffffffffu, full && same && pos - (j0 + 63) >= clamp);
+      // every pair visible and at most two time buckets per row: the position bias
+      // per pair from the shared table, the time bias switching at one column
+      const bool fastp = !fast && rp_smem && (diag || col) &&
+                         __all_sync(0xffffffffu, full && tb0 - tb1 <= 1);
       const uint32_t tcol = lane_off + 64 * g;
       if (zero) {
         uint32_t pk[8];
@@ -438,6 +443,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 8; ++e) pk[e] = 0u;
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_st8(tS + tcol + 8 * c, pk);
+      } else if (fastp) {
+        // the position bias per pair from the shared table, the time bias a row
+        // constant; position gradients along the diagonals or the columns
+        const int pos_rel = min(max(pos - kb, -1), clamp + 129);
+        // keys from column jm on have a gap below thr[tb0] (bucket tb1): the count
+        // of the half's keys with t_j <= t_i - thr[tb0] (sorted inside the user)
+        int jm = 64;
+        if (tb1 != tb0) {
+          const int64_t cut = ti - s_thr[tb0];
+          int pcount = 0;
+#pragma unroll
+          for (int step = 32; step > 0; step >>= 1)
+            if (kts[64 * g + pcount + step - 1] <= cut) pcount += step;
+          jm = pcount + (kts[64 * g + pcount] <= cut ? 1 : 0);
+        }
+        jm += 64 * g;
+        const float ht0 = s_rt[tb0], ht1 = s_rt[tb1];
+        float acc_t = 0.0f, acc_t1 = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pk[8];
+          const int jr0 = 64 * g + 16 * c;
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
+          float dsv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const bool lower = jr0 + e >= jm;
+            const float rp = s_rp[kPosPad + pos_rel - (jr0 + e)];
+            const Grad gr = silu_grad(__uint_as_float(rs[e]) + rp + (lower ? ht1 : ht0),
+                                      __uint_as_float(ra[e]), inv_nn);
+            dsv[e] = gr.ds;
+            if (lower) acc_t1 += gr.ds; else acc_t += gr.ds;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
+          tmem_st8(tS + tcol + 8 * c, pk);
+          if (diag) {
+            float acc_a = 0.0f, acc_b = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float v = __shfl_sync(0xffffffffu, dsv[e], (lane + e) & 31);
+              if (lane + e < 32) acc_a += v; else acc_b += v;
+            }
+            const int da = pos0 + lane - (kb + jr0);
+            const int db = da - 32;
+            const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
+            const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
+            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) atomicAdd(s_gpos + ba, acc_a);
+            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) atomicAdd(s_gpos + bb, acc_b);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float v = dsv[e];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              if (lane == e && v != 0.0f) {
+                const int dp = pos0 - (kb + jr0 + e);
+                const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
+                if (b == clamp) acc_c += v; else atomicAdd(s_gpos + b, v);
+              }
+            }
+          }
+        }
+        const float wsum = warp_sum(acc_t);
+        if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
+          if (lane == 0 && wsum != 0.0f) atomicAdd(s_gtime + tb0, wsum);
+        } else if (acc_t != 0.0f) {
+          atomicAdd(s_gtime + tb0, acc_t);
+        }
+        if (acc_t1 != 0.0f) atomicAdd(s_gtime + tb1, acc_t1);
       } else if (fast) {
         // every pair visible, clamped position, one time bucket per row; the
         // tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
@@ -864,29 +941,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int i0 = q0 + 64 * g;   // first query of this group's half
       // ---- classify the key row for this half tile: the half's queries' facts,
       // reduced over the warp (each lane reads two)
-      int mx_lo, mn_hi, mn_pos;
+      int mx_lo, mn_hi, mn_pos, own;   // own: every query of the half at its own index
       {
         const RowInfo fa = qf[64 * g + lane], fb = qf[64 * g + 32 + lane];
         mx_lo = max(fa.lo, fb.lo);
         mn_hi = min(fa.hi, fb.hi);
         mn_pos = min(fa.pos, fb.pos);
+        own = (fa.pos == i0 + lane && fb.pos == i0 + 32 + lane) ? 1 : 0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           mx_lo = max(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, o));
           mn_hi = min(mn_hi, __shfl_xor_sync(0xffffffffu, mn_hi, o));
           mn_pos = min(mn_pos, __shfl_xor_sync(0xffffffffu, mn_pos, o));
+          own = min(own, __shfl_xor_sync(0xffffffffu, own, o));
         }
       }
       const bool all_rows = i0 + 63 < p.T;
       const bool zero = __all_sync(0xffffffffu, !valid || i0 + 63 < j);
       const bool full = valid && all_rows && mx_lo <= j && j < mn_hi;
-      int tb0 = 0;
+      int tb0 = 0, tb1 = 0;
       bool same = false;
       if (full) {
         tb0 = bucket_search(s_thr, nb, qts[64 * g] - tj);
-        same = tb0 == bucket_search(s_thr, nb, qts[64 * g + 63] - tj);
+        tb1 = bucket_search(s_thr, nb, qts[64 * g + 63] - tj);
+        same = tb0 == tb1;
       }
       const bool fast = __all_sync(0xffffffffu, full && same && mn_pos - j >= clamp);
+      // every pair visible, one time bucket per key row, the queries at their
+      // own positions: position iq - j, read from the padded table (every pair
+      // visible keeps iq - j in [0, clamp + 95] when not all are clamped)
+      const bool fastp = !fast && own && __all_sync(0xffffffffu, full && tb1 - tb0 <= 1);
       const uint32_t tcol = lane_off + 64 * g;
       if (zero) {
         uint32_t pk[8];
@@ -896,6 +980,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < 4; ++c) {
           tmem_st8(tS + tcol + 8 * c, pk);
           tmem_st8(tdA + tcol + 8 * c, pk);
+        }
+      } else if (fastp) {
+        // queries from column im on have a gap of at least thr[tb1] (bucket tb1):
+        // the count of the half's queries with t_i < t_j + thr[tb1] (sorted)
+        int im = 64;
+        if (tb1 != tb0) {
+          const int64_t cut = tj + s_thr[tb1];
+          int pcount = 0;
+#pragma unroll
+          for (int step = 32; step > 0; step >>= 1)
+            if (qts[64 * g + pcount + step - 1] < cut) pcount += step;
+          im = pcount + (qts[64 * g + pcount] < cut ? 1 : 0);
+        }
+        const float ht0 = s_rt[tb0], ht1 = s_rt[tb1];
+        const int base = kPosPad + i0 - j;   // + column offset inside the half
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[16], ra[16], pp[8], pd[8];
+          tmem_ld16(tS + tcol + 16 * c, rs);
+          tmem_ld16(tdA + tcol + 16 * c, ra);
+          tmem_ld_wait();
+          float pv[16], dv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float rp = s_rp[min(base + 16 * c + e, kPosPad + clamp + 129)];
+            const float ht = 16 * c + e >= im ? ht1 : ht0;
+            const Grad gr = silu_grad(__uint_as_float(rs[e]) + rp + ht, __uint_as_float(ra[e]), inv_nn);
+            pv[e] = gr.p;
+            dv[e] = gr.ds;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pp[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+            pd[e] = pack_bf16x2(dv[2 * e], dv[2 * e + 1]);
+          }
+          tmem_st8(tS + tcol + 8 * c, pp);
+          tmem_st8(tdA + tcol + 8 * c, pd);
         }
       } else if (fast) {
         // the tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c

@@ -942,7 +942,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + NSK;    // [NSV] (leader)
   uint64_t* v_empty = v_full + NSV;    // [NSV]
   uint64_t* s_full = v_empty + NSV;    // [3] S buffer b holds the scores of its key tile
-  uint64_t* p_full = s_full + 3;       // [3] (leader) P written in both CTAs
+  uint64_t* p_full = s_full + 3;       // [3] (leader) P written by the scoring warps of both CTAs
   uint64_t* o_full = p_full + 3;       // every product is done
   uint64_t* drained = o_full + 1;
   uint64_t* t_full = drained + 1;      // [NST] key timestamps of a tile landed (local)
@@ -989,7 +989,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 3; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 2);   // one arrival per CTA
+      mbar_init(&p_full[b], 8);   // one arrival per row-group warp of each CTA
     }
     mbar_init(o_full, 1);
     mbar_init(drained, 1);
@@ -1124,6 +1124,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
+    // the row's facts first: their loads are in flight while the tables load
+    // (token indices fit in int32: T <= 2^30, checked at create)
+    const int i = (qt0 + q) * 128 + row;
+    const bool valid = q < nq && i < p.T;
+    int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
+    Row R;
+    R.ti = 0;
+    int64_t t_lo = 0;
+    if (valid) {
+      const RowInfo ri = p.rows[i];
+      lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
+      hi = ri.hi;
+      pos = ri.pos;
+      R.ti = p.ts[i];
+      t_lo = p.ts[lo];
+    }
+    R.ti_lo = uint32_t(R.ti);
+    const bool row_narrow = !valid || R.ti - t_lo < int64_t(0x7FFFFFFE);
     {
       // the tables, eight global loads in flight per thread before the stores
       const int t = threadIdx.x - 128;
@@ -1166,25 +1184,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     named_bar_sync(1, 256);
     const uint8_t* s_anyb = reinterpret_cast<const uint8_t*>(s_any);
 
-    // token indices fit in int32 (T <= 2^30, checked at create)
-    const int i = (qt0 + q) * 128 + row;
-    const bool valid = q < nq && i < p.T;
-    int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
-    Row R;
-    R.ti = 0;
-    if (valid) {
-      const RowInfo ri = p.rows[i];
-      lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
-      hi = ri.hi;
-      pos = ri.pos;
-      R.ti = p.ts[i];
-    }
-    R.ti_lo = uint32_t(R.ti);
-    const bool row_narrow = !valid || R.ti - p.ts[lo] < int64_t(0x7FFFFFFE);
     R.b = 0;
     R.cut = R.ti;
     if (valid) {
-      R.b = bucket_search(s_thr, nb, R.ti - p.ts[lo]);
+      R.b = bucket_search(s_thr, nb, R.ti - t_lo);
       R.cut = R.ti - s_thr[R.b];
     }
     const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
@@ -1295,11 +1298,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
         score_tile<kGen, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
       }
+      // each warp hands its 32 rows of P over on its own: no warp waits for the
+      // others of its group
       tmem_st_wait();
       tc_fence_before();
-      named_bar_sync(2 + g, 128);   // the group's P is written
-      if (wq == 0 && lane == 0) mbar_arrive_cluster(leader(&p_full[j % 3]));
-      if (lane == 0) mbar_arrive(&t_empty[st]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(leader(&p_full[j % 3]));
+        mbar_arrive(&t_empty[st]);
+      }
       if (mode == kFast || mode == kMed || mode == kCut) {
         R.b = R.b_last;
         R.cut = R.cut_last;

@@ -186,28 +186,85 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
-      if (!mbar_wait(&acc_full[acc], acc_phase, p.wait_limit)) { *abort_flag = 1; break; }
-      tc_fence_after();
       const int64_t mt = t / n_tiles;
       const int nt = int(t % n_tiles);
       const int64_t grow = mt * 128 + row;
       const bool valid = grow < p.M;   // rows past M are computed on zeros and clipped by the store
+      // fp32 residual: the loads of a chunk are issued one chunk ahead (the
+      // first chunk's before the wait for the accumulator), so that their
+      // latency overlaps the products and the previous chunk's epilogue
+      const float4* res_row = reinterpret_cast<const float4*>(
+          static_cast<const float*>(p.residual) + grow * int64_t(p.N) + nt * BN);
+      float4 xnext[8];
+      if (!out_bf16) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          xnext[e] = valid ? res_row[c_begin / 4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.wait_limit)) { *abort_flag = 1; break; }
+      tc_fence_after();
 #pragma unroll 1
       for (int c = c_begin; c < c_begin + BN / 2; c += step) {
         const int col0 = nt * BN + c;
-        // fp32 residual: issue its loads first, so that they overlap the
-        // tensor-memory read and the bias adds
-        float4 xres[8];
         if (!out_bf16) {
-          const float4* res = reinterpret_cast<const float4*>(
-              static_cast<const float*>(p.residual) + grow * int64_t(p.N) + col0);
+          // fp32 output: acc + bias + the fp32 residual (32 columns)
+          float4 xres[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xres[e] = valid ? res[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int e = 0; e < 8; ++e) xres[e] = xnext[e];
+          if (c + step < c_begin + BN / 2) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              xnext[e] = valid ? res_row[(c + step) / 4 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          uint32_t r[32];
+          tmem_ld32(tmem_base + acc * BN + c + (uint32_t(q * 32) << 16), r);
+          tmem_ld_wait();
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 bb = __ldg(b4 + e);
+            const float4 x = xres[e];
+            v[4 * e + 0] = __uint_as_float(r[4 * e + 0]) + bb.x + x.x;
+            v[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y + x.y;
+            v[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z + x.z;
+            v[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w + x.w;
+            st_shared_v4(chunk(e), v[4 * e + 0], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+          fence_proxy_async_smem();   // make the stores visible to the TMA unit
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_out, box, col0, int32_t(mt * 128 + q * 32));
+            bulk_commit_group();
+            bulk_wait_group_read0();   // the box is refilled by the next step
+          }
+          __syncwarp();
+          if (p.out_bf16) {
+            // bf16 copy of the 32 fp32 columns: 64-byte box rows, 64-byte swizzle
+            // (16-byte chunk e of row r sits at chunk e ^ ((r / 2) mod 4))
+            const uint32_t row64 = smem_u32(box + lane * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              st_shared_v4_u32(row64 + ((e ^ ((lane >> 1) & 3)) << 4),
+                               pack_bf16x2(v[8 * e + 0], v[8 * e + 1]),
+                               pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                               pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                               pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tma_out2, box, col0, int32_t(mt * 128 + q * 32));
+              bulk_commit_group();
+              bulk_wait_group_read0();
+            }
+            __syncwarp();
+          }
+          continue;
         }
+        // bf16 output (64 columns): SiLU-split, or + bias + the bf16 residual
         float v[64];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (h == 1 && !out_bf16) break;
           uint32_t r[32];
           tmem_ld32(tmem_base + acc * BN + c + 32 * h + (uint32_t(q * 32) << 16), r);
           tmem_ld_wait();
@@ -228,16 +285,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              pack_bf16x2(silu_f(v[8 * e + 2]), silu_f(v[8 * e + 3])),
                              pack_bf16x2(silu_f(v[8 * e + 4]), silu_f(v[8 * e + 5])),
                              pack_bf16x2(silu_f(v[8 * e + 6]), silu_f(v[8 * e + 7])));
-        } else if (p.io_fp32) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 x = xres[e];
-            v[4 * e + 0] += x.x;
-            v[4 * e + 1] += x.y;
-            v[4 * e + 2] += x.z;
-            v[4 * e + 3] += x.w;
-            st_shared_v4(chunk(e), v[4 * e + 0], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          }
         } else {
           const uint4* res = reinterpret_cast<const uint4*>(
               static_cast<const uint16_t*>(p.residual) + grow * int64_t(p.N) + col0);
@@ -263,26 +310,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_wait_group_read0();   // the box is refilled by the next step
         }
         __syncwarp();
-        if (!out_bf16 && p.out_bf16) {
-          // bf16 copy of the 32 fp32 columns: 64-byte box rows, 64-byte swizzle
-          // (16-byte chunk e of row r sits at chunk e ^ ((r / 2) mod 4))
-          const uint32_t row64 = smem_u32(box + lane * 64);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            st_shared_v4_u32(row64 + ((e ^ ((lane >> 1) & 3)) << 4),
-                             pack_bf16x2(v[8 * e + 0], v[8 * e + 1]),
-                             pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
-                             pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
-                             pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tma_out2, box, col0, int32_t(mt * 128 + q * 32));
-            bulk_commit_group();
-            bulk_wait_group_read0();
-          }
-          __syncwarp();
-        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
