@@ -237,8 +237,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto key_tile = [&](int j) -> int { return j < n_a ? a0 + j : qt; };
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned up to 1024 bytes by pointer arithmetic on the shared array, so that
+  // the compiler keeps every access derived from it in the shared state space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   int64_t* s_kts = reinterpret_cast<int64_t*>(smem + L::kKts);
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);
   float* s_rt = reinterpret_cast<float*>(smem + L::kRt);
@@ -492,8 +493,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int db = da - 32;
             const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
             const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
-            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) atomicAdd(s_gpos + ba, acc_a);
-            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) atomicAdd(s_gpos + bb, acc_b);
+            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) red_add_shared(s_gpos + ba, acc_a);
+            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) red_add_shared(s_gpos + bb, acc_b);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -503,18 +504,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (lane == e && v != 0.0f) {
                 const int dp = pos0 - (kb + jr0 + e);
                 const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-                if (b == clamp) acc_c += v; else atomicAdd(s_gpos + b, v);
+                if (b == clamp) acc_c += v; else red_add_shared(s_gpos + b, v);
               }
             }
           }
         }
         const float wsum = warp_sum(acc_t);
         if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
-          if (lane == 0 && wsum != 0.0f) atomicAdd(s_gtime + tb0, wsum);
+          if (lane == 0 && wsum != 0.0f) red_add_shared(s_gtime + tb0, wsum);
         } else if (acc_t != 0.0f) {
-          atomicAdd(s_gtime + tb0, acc_t);
+          red_add_shared(s_gtime + tb0, acc_t);
         }
-        if (acc_t1 != 0.0f) atomicAdd(s_gtime + tb1, acc_t1);
+        if (acc_t1 != 0.0f) red_add_shared(s_gtime + tb1, acc_t1);
       } else if (fast) {
         // every pair visible, clamped position, one time bucket per row; the
         // tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
@@ -560,9 +561,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         acc_c += acc;   // the position bucket is the clamped one for every pair here
         const float wsum = warp_sum(acc);
         if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
-          if (lane == 0 && wsum != 0.0f) atomicAdd(s_gtime + tb0, wsum);
+          if (lane == 0 && wsum != 0.0f) red_add_shared(s_gtime + tb0, wsum);
         } else if (acc != 0.0f) {
-          atomicAdd(s_gtime + tb0, acc);
+          red_add_shared(s_gtime + tb0, acc);
         }
       } else {
         // any visibility: the mask, the position bucket and the exact time bucket
@@ -616,7 +617,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int e = 0; e < 16; ++e) {
             if (tbv[e] < 0) continue;
             if (tbv[e] != run_b) {
-              if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
+              if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
               run_b = tbv[e];
               run_acc = 0.0f;
             }
@@ -636,8 +637,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int db = da - 32;
             const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
             const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
-            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) atomicAdd(s_gpos + ba, acc_a);
-            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) atomicAdd(s_gpos + bb, acc_b);
+            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) red_add_shared(s_gpos + ba, acc_a);
+            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) red_add_shared(s_gpos + bb, acc_b);
           } else if (col) {
             // one position per column: the column sums, lane e adds column e
 #pragma unroll
@@ -648,7 +649,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (lane == e && v != 0.0f) {
                 const int dp = pos0 - (kb + jr0 + e);
                 const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-                if (b == clamp) acc_c += v; else atomicAdd(s_gpos + b, v);
+                if (b == clamp) acc_c += v; else red_add_shared(s_gpos + b, v);
               }
             }
           } else {
@@ -657,11 +658,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (dsv[e] == 0.0f) continue;
               const int dp = pos - (kb + jr0 + e);
               const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-              if (b == clamp) acc_c += dsv[e]; else atomicAdd(s_gpos + b, dsv[e]);
+              if (b == clamp) acc_c += dsv[e]; else red_add_shared(s_gpos + b, dsv[e]);
             }
           }
         }
-        if (run_b >= 0 && run_acc != 0.0f) atomicAdd(s_gtime + run_b, run_acc);
+        if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -669,7 +670,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     {
       const float wsum = warp_sum(acc_c);
-      if (lane == 0 && wsum != 0.0f) atomicAdd(s_gpos + clamp, wsum);
+      if (lane == 0 && wsum != 0.0f) red_add_shared(s_gpos + clamp, wsum);
     }
     if (aborted) *abort_flag = 1;
     // ---- dQ -> the (now free) Q and dO tiles -> TMA stores; the rows past T are clipped
@@ -759,8 +760,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int nq = int((ue + 127) / 128) - kt;   // >= 1
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned up to 1024 bytes by pointer arithmetic on the shared array, so that
+  // the compiler keeps every access derived from it in the shared state space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const RowInfo* s_qf = reinterpret_cast<const RowInfo*>(smem + L::kQf);
   const int64_t* s_qts = reinterpret_cast<const int64_t*>(smem + L::kQts);
   int64_t* s_thr = reinterpret_cast<int64_t*>(smem + L::kThr);

@@ -381,6 +381,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Adds v to the fp32 word at p, which must point into this CTA's shared
+// memory (a reduction in the shared state space, whatever the compiler can
+// tell about the pointer).
+__device__ __forceinline__ void red_add_shared(float* p, float v) {
+  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
