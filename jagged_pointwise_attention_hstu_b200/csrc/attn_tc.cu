@@ -7,6 +7,10 @@
 // (same blog, section "不对序列做 softmax"), hence no running maximum and no
 // rescaling of the accumulator, and the n x n score matrix is never stored.
 //
+// Two kernels compute it.  Head dim 128 runs on the CTA-pair kernel at the end
+// of this file (clusters of two SMs, cta_group::2 products, persistent over the
+// work items); head dim 64 and the bucket-recording variant run on this one.
+//
 // One CTA computes one work item -- a pair of adjacent 128-query tiles and
 // one head -- with 12 warps:
 //   warp 0      TMA: both Q tiles once, then K tiles into an NSK-stage ring and
@@ -883,22 +887,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================ CTA-pair kernel (head dim 128)
 //
-// The same work item -- a pair of adjacent 128-query tiles and one head --
-// computed by a cluster of two CTAs on two SMs, one query tile each.  The
-// leader CTA's MMA thread issues every product of the pair with
-// cta_group::2 (M = 256: rows 0-127 from the leader's Q and tensor memory,
-// 128-255 from the peer's); K and V are split between the CTAs along the
-// products' N (each CTA loads 64 keys of K and 64 columns of V per key tile),
-// so each SM reads half of every K and V tile.  With one query tile per CTA,
-// tensor memory holds three S buffers beside O: the products of key tile
+// The same work items -- a pair of adjacent 128-query tiles and one head --
+// computed by clusters of two CTAs on two SMs, one query tile each, each
+// cluster looping over the items c, c + clusters, ... (persistent: the tables
+// load once per SM, and an item's first products run while the previous
+// item's O is read out).  The leader CTA's MMA thread issues every product
+// with cta_group::2 (M = 256: rows 0-127 from the leader's Q and tensor
+// memory, 128-255 from the peer's); K and V are split between the CTAs along
+// the products' N (each CTA loads 64 keys of K and 64 columns of V per key
+// tile), so each SM reads half of every K and V tile.  With one query tile per
+// CTA, tensor memory holds three S buffers beside O: the products of key tile
 // j + 1 and j + 2 run while the row groups score tile j, and the two row
-// groups of a CTA score alternate key tiles of its query tile.
+// groups of a CTA score alternate key tiles of its query tile.  The K, V,
+// timestamp and S rings run on one tile count across the items.
 struct PairLayout {
   static constexpr int NSK = 4, NSV = 4, NST = 4;
   static constexpr uint32_t kQ = 0;                            // 128 x 128: two 64-column boxes
   static constexpr uint32_t kK = 32768;                        // [NSK] 64 keys x 128: two 8 KB boxes
   static constexpr uint32_t kV = kK + NSK * 16384;             // [NSV] 128 keys x 64 columns
-  static constexpr uint32_t kKts = kV + NSV * 16384;           // int64 [NST][128]
+  static constexpr uint32_t kStage = kV + NSV * 16384;         // O staging: 8 warps x 4 KB
+  static constexpr uint32_t kKts = kStage + 8 * 4096;          // int64 [NST][128]
   static constexpr uint32_t kThr = kKts + NST * 1024;
   static constexpr uint32_t kThr32 = kThr + kMaxTimeBuckets * 8;
   static constexpr uint32_t kLut = kThr32 + 260 * 4;
@@ -909,10 +917,51 @@ struct PairLayout {
   static __host__ __device__ constexpr uint32_t smem_bytes(int clamp) {
     return kRabPos + ((uint32_t(clamp + 1 + 2 * kPosPad) * 4 + 15) / 16) * 16 + 1024;
   }
-  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kKts % 128 == 0, "alignment");
+  static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kStage % 1024 == 0 && kKts % 128 == 0,
+                "alignment");
   static_assert(kAnyTab % 16 == 0 && kBars % 8 == 0, "alignment");
+  // mbarriers (q_full, q_empty, the K, V and timestamp rings, s_full and p_full
+  // [3] each, o_full, o_empty, drained, p_half) and two words
+  static_assert((2 + 2 * NSK + 2 * NSV + 2 * NST + 10) * 8 + 8 <= 512, "barrier block");
 };
 static_assert(PairLayout::smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
+
+// Arrive on an mbarrier of the cluster's leader CTA from either CTA.  What it
+// hands over is tensor memory written by this thread's tcgen05.st, complete
+// (tcgen05.wait::st) and fenced (tcgen05.fence::before_thread_sync) before
+// the arrive; a cluster-scope release, which also orders every earlier memory
+// operation of the thread across the cluster, measured about 1,200 cycles per
+// arrive here, against a few tens for this one.
+__device__ __forceinline__ void arrive_leader(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// One work item of the pair kernel: head, pair, and its key tiles.
+struct PairItem {
+  int h, qt0, nq, n_a, a_lo, jb, n_kt;
+  __device__ __forceinline__ int key_tile(int j) const {
+    j += jb;
+    return j < n_a ? a_lo + j : qt0 + (j - n_a);
+  }
+};
+
+__device__ __forceinline__ PairItem pair_item(const AttnParams& p, int w) {
+  const int per_head = p.num_pairs * p.num_splits;
+  PairItem it;
+  it.h = w / per_head;
+  const int pr = p.order[(w % per_head) / p.num_splits];
+  const int split = (w % per_head) % p.num_splits;
+  it.qt0 = 2 * pr;
+  const PairTiles pt = pair_tiles(p.rows, p.T, pr);
+  it.nq = pt.n_diag;
+  it.n_a = pt.n_a;
+  it.a_lo = pt.a_lo;
+  const int n_all = pt.n_a + pt.n_diag;
+  it.jb = split * n_all / p.num_splits;
+  it.n_kt = (split + 1) * n_all / p.num_splits - it.jb;   // <= 0: nothing to do
+  return it;
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_tc_pair_kernel(const __grid_constant__ CUtensorMap tm,
@@ -936,15 +985,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   int4* s_any = reinterpret_cast<int4*>(smem + L::kAnyTab);
   int64_t* s_kts = reinterpret_cast<int64_t*>(smem + L::kKts);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* q_full = bars;             // (leader) both Q tiles landed
-  uint64_t* k_full = q_full + 1;       // [NSK] (leader) both K halves landed
+  uint64_t* q_full = bars;             // (leader) both Q tiles of an item landed
+  uint64_t* q_empty = q_full + 1;      // the item's last QK^T read Q
+  uint64_t* k_full = q_empty + 1;      // [NSK] (leader) both K halves landed
   uint64_t* k_empty = k_full + NSK;    // [NSK] the products reading the stage are done
   uint64_t* v_full = k_empty + NSK;    // [NSV] (leader)
   uint64_t* v_empty = v_full + NSV;    // [NSV]
   uint64_t* s_full = v_empty + NSV;    // [3] S buffer b holds the scores of its key tile
   uint64_t* p_full = s_full + 3;       // [3] (leader) P written by the scoring warps of both CTAs
-  uint64_t* o_full = p_full + 3;       // every product is done
-  uint64_t* drained = o_full + 1;
+  uint64_t* o_full = p_full + 3;       // every product of an item is done
+  uint64_t* o_empty = o_full + 1;      // (leader) both CTAs read O out
+  uint64_t* drained = o_empty + 1;
   uint64_t* t_full = drained + 1;      // [NST] key timestamps of a tile landed (local)
   uint64_t* t_empty = t_full + NST;    // [NST]
   uint64_t* p_half = t_empty + NST;    // arrivals of the half-tile hand-over (unused here)
@@ -952,33 +1003,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_rank();
+  const int q = int(rank);             // this CTA's query tile within each pair
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int d = p.d;
-
-  // ---- the cluster's work item (head-major, pairs longest first, then the
-  // key-range splits of a pair); this CTA's query tile is the pair's rank-th
-  const int w = blockIdx.x >> 1;
-  const int per_head = p.num_pairs * p.num_splits;
-  const int h = w / per_head;
-  const int pr = p.order[(w % per_head) / p.num_splits];
-  const int split = (w % per_head) % p.num_splits;
-  const int qt0 = 2 * pr;
-  const PairTiles pt = pair_tiles(p.rows, p.T, pr);
-  const int nq = pt.n_diag;
-  const int n_a = pt.n_a;
-  const int n_all = n_a + nq;
-  const int jb = split * n_all / p.num_splits;
-  const int n_kt = (split + 1) * n_all / p.num_splits - jb;
-  if (n_kt <= 0) return;   // uniform over the cluster: both CTAs decode the same item
-  const int q = int(rank);               // this CTA's query tile within the pair
-  auto key_tile = [&](int j) -> int {
-    j += jb;
-    return j < n_a ? pt.a_lo + j : qt0 + (j - n_a);
-  };
+  const int num_items = p.num_pairs * p.num_splits * p.H;
+  const int cid = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < NSK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -992,6 +1027,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&p_full[b], 8);   // one arrival per row-group warp of each CTA
     }
     mbar_init(o_full, 1);
+    mbar_init(o_empty, 16);       // every row-group warp of both CTAs
     mbar_init(drained, 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&t_full[s], 1);
@@ -999,8 +1035,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(p_half, 128);
     *abort_flag = 0;
-    // the leader expects both CTAs' Q tiles before the peer can issue its copy
-    if (rank == 0) mbar_arrive_expect_tx(q_full, 2 * 32768);
     fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -1022,42 +1056,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_ts);
-#pragma unroll
-      for (int b = 0; b < 2; ++b)
-        tma_load_2d_pair(smem + L::kQ + b * 16384, &tm, leader(q_full), 2 * d + h * HD + b * 64,
-                         (qt0 + q) * 128);
       int last_k[NSK], last_v[NSV];
       bool t_issued[NST];
       uint32_t t_ph[NST];
       for (int s = 0; s < NSK; ++s) last_k[s] = -1;
       for (int s = 0; s < NSV; ++s) last_v[s] = -1;
       for (int s = 0; s < NST; ++s) t_issued[s] = false, t_ph[s] = 0;
-      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
-        const int kb = key_tile(j) * 128;
-        const int s = j % NSK;
-        if (!mbar_wait(&k_empty[s], ((j / NSK) & 1) ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
-        if (rank == 0) mbar_arrive_expect_tx(&k_full[s], 2 * 16384);
+      int G = 0, n_done = 0;
+      for (int w = cid; w < num_items && !*abort_flag; w += n_clusters) {
+        const PairItem I = pair_item(p, w);
+        if (I.n_kt <= 0) continue;   // uniform over the cluster
+        // Q of this item once the previous item's last QK^T has read Q
+        if (n_done > 0 && !mbar_wait(q_empty, (n_done - 1) & 1, p.wait_limit)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (rank == 0) mbar_arrive_expect_tx(q_full, 2 * 32768);
 #pragma unroll
         for (int b = 0; b < 2; ++b)
-          tma_load_2d_pair(smem + L::kK + s * 16384 + b * 8192, &tm_k, leader(&k_full[s]),
-                           3 * d + h * HD + b * 64, kb + 64 * q);
-        last_k[s] = j;
-        const int sv = j % NSV;
-        if (!mbar_wait(&v_empty[sv], ((j / NSV) & 1) ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
-        if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * 16384);
-        tma_load_2d_pair(smem + L::kV + sv * 16384, &tm, leader(&v_full[sv]), d + h * HD + 64 * q, kb);
-        last_v[sv] = j;
-        const int st = j % NST;
-        const uint32_t tph = (j / NST) & 1;
-        if (!mbar_wait(&t_empty[st], tph ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(&t_full[st], 128 * 8);
-        tma_load_1d(s_kts + st * 128, &tm_ts, &t_full[st], kb);
-        t_issued[st] = true;
-        t_ph[st] = tph;
+          tma_load_2d_pair(smem + L::kQ + b * 16384, &tm, leader(q_full),
+                           2 * d + I.h * HD + b * 64, (I.qt0 + q) * 128);
+        bool ok = true;
+        for (int j = 0; j < I.n_kt && ok; ++j) {
+          const int g = G + j;
+          const int kb = I.key_tile(j) * 128;
+          const int s = g % NSK;
+          if (!mbar_wait(&k_empty[s], ((g / NSK) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&k_full[s], 2 * 16384);
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            tma_load_2d_pair(smem + L::kK + s * 16384 + b * 8192, &tm_k, leader(&k_full[s]),
+                             3 * d + I.h * HD + b * 64, kb + 64 * q);
+          last_k[s] = g;
+          const int sv = g % NSV;
+          if (!mbar_wait(&v_empty[sv], ((g / NSV) & 1) ^ 1, p.wait_limit)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&v_full[sv], 2 * 16384);
+          tma_load_2d_pair(smem + L::kV + sv * 16384, &tm, leader(&v_full[sv]),
+                           d + I.h * HD + 64 * q, kb);
+          last_v[sv] = g;
+          const int st = g % NST;
+          const uint32_t tph = (g / NST) & 1;
+          if (!mbar_wait(&t_empty[st], tph ^ 1, p.wait_limit)) { ok = false; break; }
+          mbar_arrive_expect_tx(&t_full[st], 128 * 8);
+          tma_load_1d(s_kts + st * 128, &tm_ts, &t_full[st], kb);
+          t_issued[st] = true;
+          t_ph[st] = tph;
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        G += I.n_kt;
+        ++n_done;
       }
       // no copy may still be in flight when the CTA ends: a stage's copies have
       // landed once the products that read it are done (the leader counts the
-      // bytes of both CTAs)
+      // bytes of both CTAs), and the last Q once the last QK^T is
       for (int s = 0; s < NSK; ++s)
         if (last_k[s] >= 0) mbar_wait(&k_empty[s], (last_k[s] / NSK) & 1);
       for (int s = 0; s < NSV; ++s)
@@ -1071,77 +1125,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16(256, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(256, HD, false, true);
       const uint32_t sQ = smem_u32(smem + L::kQ);
-      bool ok = mbar_wait(q_full, 0, p.wait_limit);
-      tc_fence_after();
-      // S_j = Q K_j^T into buffer j % 3 (the K stage is released when it is done)
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % NSK;
-        if (!mbar_wait(&k_full[s], (j / NSK) & 1, p.wait_limit)) return false;
+      bool ok = true;
+      int G = 0, n_done = 0;
+      for (int w = cid; ok && w < num_items && !*abort_flag; w += n_clusters) {
+        const PairItem I = pair_item(p, w);
+        if (I.n_kt <= 0) continue;
+        if (!mbar_wait(q_full, n_done & 1, p.wait_limit)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(smem + L::kK + s * 16384);
+        // S of the item's tile j = Q K^T into buffer (G + j) % 3, after the products
+        // issued before it (in order): the K stage is released when it is done, Q
+        // after the item's last one
+        auto issue_s = [&](int j) -> bool {
+          const int g = G + j;
+          const int s = g % NSK;
+          if (!mbar_wait(&k_full[s], (g / NSK) & 1, p.wait_limit)) return false;
+          tc_fence_after();
+          const uint32_t sK = smem_u32(smem + L::kK + s * 16384);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t ok2 = (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_ss_pair(tS(j % 3), desc_sw128(sQ + oq, 16, 1024), desc_sw128(sK + ok2, 16, 1024),
-                       idesc_qk, kk > 0);
-        }
-        umma_commit_pair(&s_full[j % 3]);
-        umma_commit_pair(&k_empty[s]);
-        return true;
-      };
-      for (int j = 0; ok && j < 3 && j < n_kt; ++j) ok = issue_s(j);
-      bool o_done = false;
-      for (int j = 0; ok && j < n_kt; ++j) {
-        const int b = j % 3;
-        const int sv = j % NSV;
-        if (!mbar_wait(&p_full[b], (j / 3) & 1, p.wait_limit)) { ok = false; break; }
-        if (!mbar_wait(&v_full[sv], (j / NSV) & 1, p.wait_limit)) { ok = false; break; }
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t oq = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t ok2 = (kk >> 2) * 8192 + (kk & 3) * 32;
+            umma_ss_pair(tS(g % 3), desc_sw128(sQ + oq, 16, 1024), desc_sw128(sK + ok2, 16, 1024),
+                         idesc_qk, kk > 0);
+          }
+          umma_commit_pair(&s_full[g % 3]);
+          umma_commit_pair(&k_empty[s]);
+          if (j + 1 == I.n_kt) umma_commit_pair(q_empty);
+          return true;
+        };
+        for (int j = 0; ok && j < 3 && j < I.n_kt; ++j) ok = issue_s(j);
+        // O is rewritten from zero only after both CTAs read the previous item's O
+        if (ok && n_done > 0 && !mbar_wait(o_empty, (n_done - 1) & 1, p.wait_limit)) ok = false;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + L::kV + sv * 16384);
+        for (int j = 0; ok && j < I.n_kt; ++j) {
+          const int g = G + j;
+          const int b = g % 3;
+          const int sv = g % NSV;
+          if (!mbar_wait(&p_full[b], (g / 3) & 1, p.wait_limit)) { ok = false; break; }
+          if (!mbar_wait(&v_full[sv], (g / NSV) & 1, p.wait_limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sV = smem_u32(smem + L::kV + sv * 16384);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts_pair(tO, tS(b) + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
-                       (j > 0 || kk > 0));
-        umma_commit_pair(&v_empty[sv]);
-        if (j + 1 == n_kt) {
-          umma_commit_pair(o_full);
-          o_done = true;
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts_pair(tO, tS(b) + kk * 8, desc_sw128(sV + kk * 2048, 16384, 1024), idesc_pv,
+                         (j > 0 || kk > 0));
+          umma_commit_pair(&v_empty[sv]);
+          if (j + 1 == I.n_kt) umma_commit_pair(o_full);
+          // buffer b is rewritten only after P_j V_j (issued just above, executed in order)
+          if (j + 3 < I.n_kt && !issue_s(j + 3)) ok = false;
         }
-        // buffer b is rewritten only after P_j V_j (issued just above, executed in order)
-        if (j + 3 < n_kt && !issue_s(j + 3)) ok = false;
+        G += I.n_kt;
+        ++n_done;
       }
       if (!ok) *abort_flag = 1;
-      if (!o_done) umma_commit_pair(o_full);   // release the row groups on an abort
-      umma_commit_pair(drained);
+      umma_commit_pair(drained);   // fires once every product issued here is done
       mbar_wait(drained, 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ row groups
-    const int g = (warp - 4) >> 2;             // this group scores key tiles j = g, g + 2, ...
+    const int g = (warp - 4) >> 2;             // this group scores an item's key tiles j = g, g + 2, ...
     const int wq = warp & 3;                   // tensor-memory lane quarter
     const int row = wq * 32 + lane;
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const int clamp = p.pos_clamp;
     const int nb = p.time_buckets;
-    // the row's facts first: their loads are in flight while the tables load
-    // (token indices fit in int32: T <= 2^30, checked at create)
-    const int i = (qt0 + q) * 128 + row;
-    const bool valid = q < nq && i < p.T;
-    int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
-    Row R;
-    R.ti = 0;
-    int64_t t_lo = 0;
-    if (valid) {
-      const RowInfo ri = p.rows[i];
-      lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
-      hi = ri.hi;
-      pos = ri.pos;
-      R.ti = p.ts[i];
-      t_lo = p.ts[lo];
-    }
-    R.ti_lo = uint32_t(R.ti);
-    const bool row_narrow = !valid || R.ti - t_lo < int64_t(0x7FFFFFFE);
     {
       // the tables, eight global loads in flight per thread before the stores
       const int t = threadIdx.x - 128;
@@ -1183,13 +1230,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     named_bar_sync(1, 256);
     const uint8_t* s_anyb = reinterpret_cast<const uint8_t*>(s_any);
-
-    R.b = 0;
-    R.cut = R.ti;
-    if (valid) {
-      R.b = bucket_search(s_thr, nb, R.ti - t_lo);
-      R.cut = R.ti - s_thr[R.b];
-    }
     const int nn = p.n_norm_fixed > 0 ? p.n_norm_fixed : p.counters[0];
     const float inv_nn = 1.0f / float(nn > 0 ? nn : 1);
     Record rec;
@@ -1197,156 +1237,195 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     rec.tidx = nullptr;
     rec.vis = nullptr;
     rec.T = p.T;
-    rec.i = i;
     rec.kb = 0;
     rec.on = false;
     bool aborted = false;
+    int G = 0, n_done = 0;
 
-    for (int j = g; j < n_kt; j += 2) {
-      const int kb = key_tile(j) * 128;
-      const int st = j % NST;
-      const int64_t* kts = s_kts + st * 128;
-      bool ok = aborted ? false : mbar_wait(&t_full[st], (j / NST) & 1, p.wait_limit);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        aborted = true;
-        *abort_flag = 1;
-        break;
+    for (int w = cid; w < num_items && !aborted && !*abort_flag; w += n_clusters) {
+      const PairItem I = pair_item(p, w);
+      if (I.n_kt <= 0) continue;
+      // the row's facts (token indices fit in int32: T <= 2^30, checked at create)
+      const int i = (I.qt0 + q) * 128 + row;
+      const bool valid = q < I.nq && i < p.T;
+      int lo = 0, hi = 0, pos = 0;   // rows past T see nothing
+      Row R;
+      R.ti = 0;
+      int64_t t_lo = 0;
+      if (valid) {
+        const RowInfo ri = p.rows[i];
+        lo = (ri.lo < 0 || ri.lo > i) ? i : ri.lo;
+        hi = ri.hi;
+        pos = ri.pos;
+        R.ti = p.ts[i];
+        t_lo = p.ts[lo];
       }
-      // ---- classify this row for the tile
-      R.lo_rel = min(max(lo - kb, -1), 129);
-      R.hi_rel = min(max(hi - kb, -1), 129);
-      R.i_rel = valid ? min(max(i - kb, -1), 129) : -1;
-      R.pos_rel = min(max(pos - kb, -1), clamp + 129);
-      const bool full = valid && lo <= kb && hi - kb >= 128;
-      const bool posc = pos - kb - 127 >= clamp;
-      int lev = 99;
-      if (full) {
-        walk_to(R.b, R.cut, kts[0], R.ti, s_thr);
-        R.b_last = R.b;
-        R.cut_last = R.cut;
-        walk_to(R.b_last, R.cut_last, kts[127], R.ti, s_thr);
-        lev = R.b - R.b_last;
+      R.ti_lo = uint32_t(R.ti);
+      const bool row_narrow = !valid || R.ti - t_lo < int64_t(0x7FFFFFFE);
+      R.b = 0;
+      R.cut = R.ti;
+      if (valid) {
+        R.b = bucket_search(s_thr, nb, R.ti - t_lo);
+        R.cut = R.ti - s_thr[R.b];
       }
-      int mode;
-      if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
-      else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
-      else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
-      else if (__all_sync(0xffffffffu, full && lev <= 3)) mode = kCut;
-      else if (__all_sync(0xffffffffu, !valid || hi <= kb))
-        mode = kSelf;  // candidates on their own tiles: only the row itself is visible
-      else if (p.lut_exact && __all_sync(0xffffffffu, row_narrow))
-        mode = kAny;   // the causal diagonal, user and history boundaries, candidates
-      else mode = kGen;
-      const bool pc = __all_sync(0xffffffffu, posc);
-      if (mode == kFast || mode == kMed || mode == kCut) {
-        // R.b = bucket of the tile's first key (the largest gap); a gap below
-        // thr[R.b - m + 1] drops the bucket below R.b - m + 1
-        const float rp_c = pc ? s_rab_pos[kPosPad + clamp] : 0.0f;
-        const int b0 = R.b;
-        R.hc = 0.5f * (rp_c + s_rab_time[b0]);
-        R.hc_lo = 0.5f * (rp_c + s_rab_time[max(b0 - 1, 0)]);
-        R.hc2 = 0.5f * (rp_c + s_rab_time[max(b0 - 2, 0)]);
-        R.hc3 = 0.5f * (rp_c + s_rab_time[max(b0 - 3, 0)]);
-        if (mode != kFast) {
-          // first column whose gap is below thr[b0 - m + 1]: the count of keys with
-          // t_j <= t_i - thr[b0 - m + 1] (the tile's timestamps are sorted)
-          const int64_t c1 = R.ti - s_thr[b0];
-          const int64_t c2 = R.ti - s_thr[max(b0 - 1, 0)];
-          const int64_t c3 = R.ti - s_thr[max(b0 - 2, 0)];
-          int p1 = 0, p2 = 0, p3 = 0;
-#pragma unroll
-          for (int step = 64; step > 0; step >>= 1) {
-            if (kts[p1 + step - 1] <= c1) p1 += step;
-            if (mode == kCut) {
-              if (kts[p2 + step - 1] <= c2) p2 += step;
-              if (kts[p3 + step - 1] <= c3) p3 += step;
-            }
-          }
-          // seven halvings leave p in [0, 127]; one more compare completes the count
-          R.j1 = p1 + (kts[p1] <= c1 ? 1 : 0);
-          R.j2 = p2 + (kts[p2] <= c2 ? 1 : 0);
-          R.j3 = p3 + (kts[p3] <= c3 ? 1 : 0);
+      rec.i = i;
+
+      for (int j = g; j < I.n_kt; j += 2) {
+        const int gt = G + j;
+        const int kb = I.key_tile(j) * 128;
+        const int st = gt % NST;
+        const int64_t* kts = s_kts + st * 128;
+        bool ok = mbar_wait(&t_full[st], (gt / NST) & 1, p.wait_limit);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          aborted = true;
+          *abort_flag = 1;
+          break;
         }
-      }
-      ok = mbar_wait(&s_full[j % 3], (j / 3) & 1, p.wait_limit);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        aborted = true;
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tS(j % 3) + lane_off;
-      // rp_row[-column] = rab_pos[clamp(pos_rel - column, 0, clamp)]
-      const float* rp_row = s_rab_pos + kPosPad + R.pos_rel;
-      if (mode == kZero) {
-        zero_tile<RECORD>(taddr, rec);
-      } else if (mode == kSelf) {
-        self_tile<RECORD>(taddr, R, rp_row, s_rab_time, clamp, rec);
-      } else if (mode == kFast) {
-        if (pc) score_tile<kFast, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-        else score_tile<kFast, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-      } else if (mode == kMed) {
-        if (pc) score_tile<kMed, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-        else score_tile<kMed, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-      } else if (mode == kCut) {
-        if (pc) score_tile<kCut, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-        else score_tile<kCut, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-      } else if (mode == kAny) {
-        score_tile<kAny, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-      } else {
-        score_tile<kGen, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
-      }
-      // each warp hands its 32 rows of P over on its own: no warp waits for the
-      // others of its group
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(leader(&p_full[j % 3]));
-        mbar_arrive(&t_empty[st]);
-      }
-      if (mode == kFast || mode == kMed || mode == kCut) {
-        R.b = R.b_last;
-        R.cut = R.cut_last;
-      }
-    }
-
-    // ---- O / n_norm -> the (now free) Q tile, 32 columns per warp and pass,
-    // group g columns [64 g, 64 g + 64) -> TMA stores (or reductions into a
-    // zeroed O when the pair's key range is split)
-    bool ok = aborted ? false : mbar_wait(o_full, 0, p.wait_limit);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && q < nq) {
-      tc_fence_after();
-      uint8_t* stage = smem + L::kQ + (g * 4 + wq) * 4096;
-#pragma unroll 1
-      for (int rd = 0; rd < 2; ++rd) {
-        const int col = 64 * g + 32 * rd;
-        uint32_t r[32];
-        tmem_ld32(tO + lane_off + col, r);
-        tmem_ld_wait();
-        const uint32_t row_addr = smem_u32(stage + lane * 128);
+        // ---- classify this row for the tile
+        R.lo_rel = min(max(lo - kb, -1), 129);
+        R.hi_rel = min(max(hi - kb, -1), 129);
+        R.i_rel = valid ? min(max(i - kb, -1), 129) : -1;
+        R.pos_rel = min(max(pos - kb, -1), clamp + 129);
+        const bool full = valid && lo <= kb && hi - kb >= 128;
+        const bool posc = pos - kb - 127 >= clamp;
+        int lev = 99;
+        if (full) {
+          walk_to(R.b, R.cut, kts[0], R.ti, s_thr);
+          R.b_last = R.b;
+          R.cut_last = R.cut;
+          walk_to(R.b_last, R.cut_last, kts[127], R.ti, s_thr);
+          lev = R.b - R.b_last;
+        }
+        int mode;
+        if (__all_sync(0xffffffffu, R.i_rel < 0)) mode = kZero;   // every key is later than every row
+        else if (__all_sync(0xffffffffu, full && lev == 0)) mode = kFast;
+        else if (__all_sync(0xffffffffu, full && lev <= 1)) mode = kMed;
+        else if (__all_sync(0xffffffffu, full && lev <= 3)) mode = kCut;
+        else if (__all_sync(0xffffffffu, !valid || hi <= kb))
+          mode = kSelf;  // candidates on their own tiles: only the row itself is visible
+        else if (p.lut_exact && __all_sync(0xffffffffu, row_narrow))
+          mode = kAny;   // the causal diagonal, user and history boundaries, candidates
+        else mode = kGen;
+        const bool pc = __all_sync(0xffffffffu, posc);
+        if (mode == kFast || mode == kMed || mode == kCut) {
+          // R.b = bucket of the tile's first key (the largest gap); a gap below
+          // thr[R.b - m + 1] drops the bucket below R.b - m + 1
+          const float rp_c = pc ? s_rab_pos[kPosPad + clamp] : 0.0f;
+          const int b0 = R.b;
+          R.hc = 0.5f * (rp_c + s_rab_time[b0]);
+          R.hc_lo = 0.5f * (rp_c + s_rab_time[max(b0 - 1, 0)]);
+          R.hc2 = 0.5f * (rp_c + s_rab_time[max(b0 - 2, 0)]);
+          R.hc3 = 0.5f * (rp_c + s_rab_time[max(b0 - 3, 0)]);
+          if (mode != kFast) {
+            // first column whose gap is below thr[b0 - m + 1]: the count of keys with
+            // t_j <= t_i - thr[b0 - m + 1] (the tile's timestamps are sorted)
+            const int64_t c1 = R.ti - s_thr[b0];
+            const int64_t c2 = R.ti - s_thr[max(b0 - 1, 0)];
+            const int64_t c3 = R.ti - s_thr[max(b0 - 2, 0)];
+            int p1 = 0, p2 = 0, p3 = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4), __uint_as_float(r[4 * e + 0]) * inv_nn,
-                       __uint_as_float(r[4 * e + 1]) * inv_nn, __uint_as_float(r[4 * e + 2]) * inv_nn,
-                       __uint_as_float(r[4 * e + 3]) * inv_nn);
-        fence_proxy_async_smem();
+            for (int step = 64; step > 0; step >>= 1) {
+              if (kts[p1 + step - 1] <= c1) p1 += step;
+              if (mode == kCut) {
+                if (kts[p2 + step - 1] <= c2) p2 += step;
+                if (kts[p3 + step - 1] <= c3) p3 += step;
+              }
+            }
+            // seven halvings leave p in [0, 127]; one more compare completes the count
+            R.j1 = p1 + (kts[p1] <= c1 ? 1 : 0);
+            R.j2 = p2 + (kts[p2] <= c2 ? 1 : 0);
+            R.j3 = p3 + (kts[p3] <= c3 ? 1 : 0);
+          }
+        }
+        ok = mbar_wait(&s_full[gt % 3], (gt / 3) & 1, p.wait_limit);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          aborted = true;
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tS(gt % 3) + lane_off;
+        // rp_row[-column] = rab_pos[clamp(pos_rel - column, 0, clamp)]
+        const float* rp_row = s_rab_pos + kPosPad + R.pos_rel;
+        if (mode == kZero) {
+          zero_tile<RECORD>(taddr, rec);
+        } else if (mode == kSelf) {
+          self_tile<RECORD>(taddr, R, rp_row, s_rab_time, clamp, rec);
+        } else if (mode == kFast) {
+          if (pc) score_tile<kFast, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+          else score_tile<kFast, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+        } else if (mode == kMed) {
+          if (pc) score_tile<kMed, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+          else score_tile<kMed, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+        } else if (mode == kCut) {
+          if (pc) score_tile<kCut, true, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+          else score_tile<kCut, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+        } else if (mode == kAny) {
+          score_tile<kAny, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+        } else {
+          score_tile<kGen, false, RECORD>(taddr, R, rp_row, s_rab_time, s_thr, s_anyb, s_thr32, kts, clamp, rec, p_half);
+        }
+        // each warp hands its 32 rows of P over on its own: no warp waits for the
+        // others of its group
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          const int32_t x = h * HD + col;
-          const int32_t y = (qt0 + q) * 128 + wq * 32;
-          if (p.num_splits > 1) tma_reduce_add_2d(&tm_o, stage, x, y);
-          else tma_store_2d(&tm_o, stage, x, y);
-          bulk_commit_group();
-          bulk_wait_group_read0();
+          arrive_leader(leader(&p_full[gt % 3]));
+          mbar_arrive(&t_empty[st]);
         }
-        __syncwarp();
+        if (mode == kFast || mode == kMed || mode == kCut) {
+          R.b = R.b_last;
+          R.cut = R.cut_last;
+        }
       }
-    } else if (!ok) {
-      *abort_flag = 1;
+      if (aborted) break;
+
+      // ---- O / n_norm -> staging (32 columns per warp and pass, group g columns
+      // [64 g, 64 g + 64)) -> TMA stores, or reductions into a zeroed O when the
+      // pair's key range is split; then O's columns are released to the next item
+      bool ok = mbar_wait(o_full, n_done & 1, p.wait_limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        aborted = true;
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      if (q < I.nq) {
+        uint8_t* stage = smem + L::kStage + (g * 4 + wq) * 4096;
+#pragma unroll 1
+        for (int rd = 0; rd < 2; ++rd) {
+          const int col = 64 * g + 32 * rd;
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + col, r);
+          tmem_ld_wait();
+          const uint32_t row_addr = smem_u32(stage + lane * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            st_shared_v4(row_addr + ((e ^ (lane & 7)) << 4), __uint_as_float(r[4 * e + 0]) * inv_nn,
+                         __uint_as_float(r[4 * e + 1]) * inv_nn, __uint_as_float(r[4 * e + 2]) * inv_nn,
+                         __uint_as_float(r[4 * e + 3]) * inv_nn);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int32_t x = I.h * HD + col;
+            const int32_t y = (I.qt0 + q) * 128 + wq * 32;
+            if (p.num_splits > 1) tma_reduce_add_2d(&tm_o, stage, x, y);
+            else tma_store_2d(&tm_o, stage, x, y);
+            bulk_commit_group();
+            bulk_wait_group_read0();   // the box is reused by the next pass or item
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_leader(leader(o_empty));
+      G += I.n_kt;
+      ++n_done;
     }
   }
 
@@ -1420,8 +1499,8 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
     if (ez != cudaSuccess) return ez;
   }
   const int64_t grid = int64_t(a.num_pairs) * a.H * p.num_splits;
-  if (HD == 128 && !RECORD && a.use_pair) {
-    // one CTA pair per work item: K halves come through their own tensor map
+  if (HD == 128 && !RECORD) {
+    // CTA pairs: K halves come through their own tensor map
     if (!make_tmap_2d_bf16(&tm_k, a.uvqk, uint64_t(4 * a.d), uint64_t(a.T), uint64_t(4 * a.d) * 2,
                            64, 64))
       return cudaErrorInvalidValue;
@@ -1429,8 +1508,13 @@ cudaError_t launch_hd(const AttnArgs& a, cudaStream_t st) {
     const cudaError_t ep = smem_opt_in(attn_tc_pair_kernel,
                                        int(PairLayout::smem_bytes(kMaxPosEntries - 1)), pair_set);
     if (ep != cudaSuccess) return ep;
-    attn_tc_pair_kernel<<<unsigned(2 * grid), kThreads, PairLayout::smem_bytes(a.pos_clamp), st>>>(
-        tm, tm_k, tm_ts, tm_o, p);
+    // persistent: one cluster per two SMs (or per item, when there are fewer)
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t clusters = grid < sms / 2 ? grid : int64_t(sms / 2 > 0 ? sms / 2 : 1);
+    attn_tc_pair_kernel<<<unsigned(2 * clusters), kThreads, PairLayout::smem_bytes(a.pos_clamp),
+                          st>>>(tm, tm_k, tm_ts, tm_o, p);
     return cudaGetLastError();
   }
   attn_tc_kernel<HD, RECORD><<<unsigned(grid), kThreads, L::smem_bytes(a.pos_clamp), st>>>(tm, tm_ts, tm_o, p);

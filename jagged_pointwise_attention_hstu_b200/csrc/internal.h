@@ -233,7 +233,6 @@ struct AttnArgs {
   int lut_exact;             // time_log_div > ln 1.25: the candidate-bucket table is exact
   int64_t wait_limit;        // bound of the pipeline waits in SM cycles (0: the default)
   int64_t q_row0;            // first row of the listed pairs (rows [q_row0, T) are written)
-  int use_pair;              // head dim 128: one CTA pair (cta_group::2) per work item
   // recording variant
   int32_t* dump_pidx;
   int32_t* dump_tidx;
