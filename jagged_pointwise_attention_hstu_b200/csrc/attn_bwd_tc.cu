@@ -462,13 +462,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         jm += 64 * g;
         const float ht0 = s_rt[tb0], ht1 = s_rt[tb1];
         float acc_t = 0.0f, acc_t1 = 0.0f;
+        // the next chunk's tensor-memory loads run under this chunk's reductions
+        uint32_t rs[16], ra[16];
+        tmem_ld16(tS + tcol, rs);
+        tmem_ld16(tdA + tcol, ra);
+        tmem_ld_wait();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pk[8];
+          uint32_t pk[8];
           const int jr0 = 64 * g + 16 * c;
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
           float dsv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -482,6 +484,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
           tmem_st8(tS + tcol + 8 * c, pk);
+          if (c + 1 < 4) {
+            tmem_ld16(tS + tcol + 16 * (c + 1), rs);
+            tmem_ld16(tdA + tcol + 16 * (c + 1), ra);
+          }
           if (diag) {
             float acc_a = 0.0f, acc_b = 0.0f;
 #pragma unroll
@@ -508,6 +514,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               }
             }
           }
+          tmem_ld_wait();
         }
         const float wsum = warp_sum(acc_t);
         if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
@@ -575,13 +582,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int pos_rel = min(max(pos - kb, -1), clamp + 129);
         int run_b = -1;
         float run_acc = 0.0f;
+        uint32_t rs[16], ra[16];
+        tmem_ld16(tS + tcol, rs);
+        tmem_ld16(tdA + tcol, ra);
+        tmem_ld_wait();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pk[8];
+          uint32_t pk[8];
           const int jr0 = 64 * g + 16 * c;
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
           float dsv[16];
           int tbv[16];
 #pragma unroll
@@ -612,16 +620,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = pack_bf16x2(dsv[2 * e], dsv[2 * e + 1]);
           tmem_st8(tS + tcol + 8 * c, pk);
-          // time buckets: runs of one bucket along the row
+          if (c + 1 < 4) {   // the next chunk's loads run under this chunk's reductions
+            tmem_ld16(tS + tcol + 16 * (c + 1), rs);
+            tmem_ld16(tdA + tcol + 16 * (c + 1), ra);
+          }
+          // time buckets: runs of one bucket along the row, without branches (a
+          // run's sum is added when a visible pair of another bucket starts the next)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            if (tbv[e] < 0) continue;
-            if (tbv[e] != run_b) {
-              if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
-              run_b = tbv[e];
-              run_acc = 0.0f;
-            }
-            run_acc += dsv[e];
+            const bool next = tbv[e] >= 0 && tbv[e] != run_b;
+            red_add_shared_if(next && run_b >= 0, s_gtime + (run_b < 0 ? 0 : run_b), run_acc);
+            run_acc = next ? dsv[e] : run_acc + dsv[e];
+            run_b = next ? tbv[e] : run_b;
           }
           // position buckets
           if (diag) {
@@ -661,6 +671,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               if (b == clamp) acc_c += dsv[e]; else red_add_shared(s_gpos + b, dsv[e]);
             }
           }
+          tmem_ld_wait();
         }
         if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
       }
@@ -997,12 +1008,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float ht0 = s_rt[tb0], ht1 = s_rt[tb1];
         const int base = kPosPad + i0 - j;   // + column offset inside the half
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pp[8], pd[8];
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
+        auto chunk = [&](const uint32_t (&rs)[16], const uint32_t (&ra)[16], int c) {
+          uint32_t pp[8], pd[8];
           float pv[16], dv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -1019,6 +1026,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tmem_st8(tS + tcol + 8 * c, pp);
           tmem_st8(tdA + tcol + 8 * c, pd);
+        };
+        // the tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
+        uint32_t xs[16], xa[16], ys[16], ya[16];
+        tmem_ld16(tS + tcol, xs);
+        tmem_ld16(tdA + tcol, xa);
+        tmem_ld_wait();
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld16(tS + tcol + 16 * (c + 1), ys);
+          tmem_ld16(tdA + tcol + 16 * (c + 1), ya);
+          chunk(xs, xa, c);
+          tmem_ld_wait();
+          if (c + 2 < 4) {
+            tmem_ld16(tS + tcol + 16 * (c + 2), xs);
+            tmem_ld16(tdA + tcol + 16 * (c + 2), xa);
+          }
+          chunk(ys, ya, c + 1);
+          tmem_ld_wait();
         }
       } else if (fast) {
         // the tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
@@ -1063,12 +1088,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_wait();
         }
       } else {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rs[16], ra[16], pp[8], pd[8];
-          tmem_ld16(tS + tcol + 16 * c, rs);
-          tmem_ld16(tdA + tcol + 16 * c, ra);
-          tmem_ld_wait();
+        auto chunk = [&](const uint32_t (&rs)[16], const uint32_t (&ra)[16], int c) {
+          uint32_t pp[8], pd[8];
           float pv[16], dv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -1099,6 +1120,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tmem_st8(tS + tcol + 8 * c, pp);
           tmem_st8(tdA + tcol + 8 * c, pd);
+        };
+        // the tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
+        uint32_t xs[16], xa[16], ys[16], ya[16];
+        tmem_ld16(tS + tcol, xs);
+        tmem_ld16(tdA + tcol, xa);
+        tmem_ld_wait();
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld16(tS + tcol + 16 * (c + 1), ys);
+          tmem_ld16(tdA + tcol + 16 * (c + 1), ya);
+          chunk(xs, xa, c);
+          tmem_ld_wait();
+          if (c + 2 < 4) {
+            tmem_ld16(tS + tcol + 16 * (c + 2), xs);
+            tmem_ld16(tdA + tcol + 16 * (c + 2), xa);
+          }
+          chunk(ys, ya, c + 1);
+          tmem_ld_wait();
         }
       }
       tmem_st_wait();

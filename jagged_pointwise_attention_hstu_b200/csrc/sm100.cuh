@@ -388,6 +388,16 @@ __device__ __forceinline__ void red_add_shared(float* p, float v) {
   asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
 }
 
+// The same, done only where `pred` holds: a predicated instruction, so that a
+// per-lane condition costs no divergent branch.
+__device__ __forceinline__ void red_add_shared_if(bool pred, float* p, float v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q red.shared.add.f32 [%0], %1;\n\t}" ::"r"(
+          smem_u32(p)),
+      "f"(v), "r"(int(pred))
+      : "memory");
+}
+
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
