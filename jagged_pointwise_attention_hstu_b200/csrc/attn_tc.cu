@@ -926,17 +926,6 @@ struct PairLayout {
 };
 static_assert(PairLayout::smem_bytes(kMaxPosEntries - 1) <= 227 * 1024, "shared memory budget");
 
-// Arrive on an mbarrier of the cluster's leader CTA from either CTA.  What it
-// hands over is tensor memory written by this thread's tcgen05.st, complete
-// (tcgen05.wait::st) and fenced (tcgen05.fence::before_thread_sync) before
-// the arrive; a cluster-scope release, which also orders every earlier memory
-// operation of the thread across the cluster, measured about 1,200 cycles per
-// arrive here, against a few tens for this one.
-__device__ __forceinline__ void arrive_leader(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 // One work item of the pair kernel: head, pair, and its key tiles.
 struct PairItem {
   int h, qt0, nq, n_a, a_lo, jb, n_kt;

@@ -29,7 +29,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 4;
 constexpr int kBK = 64;   // one 128-byte swizzle row of bf16
 
 struct GemmParams {
@@ -45,10 +44,13 @@ struct GemmParams {
   int32_t* error;
 };
 
-template <int BN>
+// PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
+// products (each CTA holds 128 rows of A and BN / 2 rows of the B tile).
+template <int BN, bool PAIR>
 struct GemmLayout {
+  static constexpr int kStages = PAIR ? 6 : 4;
   static constexpr uint32_t kABytes = 128 * kBK * 2;
-  static constexpr uint32_t kBBytes = BN * kBK * 2;
+  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kOutOffset = kStages * kStageBytes;   // 8 boxes of 4 KB
   static constexpr uint32_t kBarOffset = kOutOffset + 8 * 4096;
@@ -64,13 +66,12 @@ __device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + _
 
 constexpr int kGemmThreads = 320;
 
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
-                   const __grid_constant__ CUtensorMap tma_b,
-                   const __grid_constant__ CUtensorMap tma_out,
-                   const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
-  using L = GemmLayout<BN>;
+template <int BN, bool PAIR>
+__device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
+                                          const CUtensorMap* tma_out, const CUtensorMap* tma_out2,
+                                          const GemmParams& p) {
+  using L = GemmLayout<BN, PAIR>;
+  constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,6 +85,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // PAIR: this CTA's half of the cluster's 256-row tile; the leader (rank 0)
+  // counts both CTAs' loads and epilogue releases and issues every product
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  auto leader = [&](uint64_t* bar) -> uint32_t { return map_to_rank(smem_u32(bar), 0); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -92,29 +97,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 256);
+      mbar_init(&acc_empty[a], PAIR ? 16 : 256);   // PAIR: each epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * BN);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, 2 * BN);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 2 * BN);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tma_a);
-    prefetch_tmap(&tma_b);
+    prefetch_tmap(tma_a);
+    prefetch_tmap(tma_b);
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the leader's barriers exist before the peer's loads signal them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t m_tiles = (p.M + 127) / 128;
+  constexpr int kTileM = PAIR ? 256 : 128;
+  const int64_t m_tiles = (p.M + kTileM - 1) / kTileM;
   const int n_tiles = p.N / BN;
   const int64_t total = m_tiles * n_tiles;
   const int kblocks = p.K / kBK;
+  const int64_t t0 = PAIR ? int64_t(blockIdx.x >> 1) : int64_t(blockIdx.x);
+  const int64_t t_step = PAIR ? int64_t(gridDim.x >> 1) : int64_t(gridDim.x);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -122,30 +136,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_phase[kStages];
       bool issued[kStages];
       for (int s = 0; s < kStages; ++s) issued[s] = false, issued_phase[s] = 0;
-      for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      for (int64_t t = t0; t < total && !*abort_flag; t += t_step) {
         const int64_t mt = t / n_tiles;
         const int nt = int(t % n_tiles);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
-          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
           uint8_t* sa = smem + stage * L::kStageBytes;
-          tma_load_2d(sa, &tma_a, &full[stage], kb * kBK, int32_t(mt * 128));
-          tma_load_2d(sa + L::kABytes, &tma_b, &full[stage], kb * kBK, nt * BN);
+          if constexpr (PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStageBytes);
+            tma_load_2d_pair(sa, tma_a, leader(&full[stage]), kb * kBK,
+                             int32_t(mt * 256 + rank * 128));
+            tma_load_2d_pair(sa + L::kABytes, tma_b, leader(&full[stage]), kb * kBK,
+                             nt * BN + int(rank) * (BN / 2));
+          } else {
+            mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+            tma_load_2d(sa, tma_a, &full[stage], kb * kBK, int32_t(mt * 128));
+            tma_load_2d(sa + L::kABytes, tma_b, &full[stage], kb * kBK, nt * BN);
+          }
           issued[stage] = true;
           issued_phase[stage] = phase;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
       }
-      // every load this thread issued has landed before the CTA may exit
+      // every load this thread issued has landed before the CTA may exit (PAIR:
+      // the leader counts them, so wait for the products that read the stage)
       for (int s = 0; s < kStages; ++s)
-        if (issued[s]) mbar_wait(&full[s], issued_phase[s]);
+        if (issued[s]) {
+          if constexpr (PAIR) mbar_wait(&empty[s], issued_phase[s]);
+          else mbar_wait(&full[s], issued_phase[s]);
+        }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, BN, false, false);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, BN, false, false);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool any = false;
-      for (int64_t t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      for (int64_t t = t0; t < total && !*abort_flag; t += t_step) {
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, p.wait_limit)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -156,18 +182,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_addr = a_addr + L::kABytes;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            umma_ss(d_tmem, desc_sw128(a_addr + k * 32, 16, 1024),
-                    desc_sw128(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+            if constexpr (PAIR)
+              umma_ss_pair(d_tmem, desc_sw128(a_addr + k * 32, 16, 1024),
+                           desc_sw128(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
+            else
+              umma_ss(d_tmem, desc_sw128(a_addr + k * 32, 16, 1024),
+                      desc_sw128(b_addr + k * 32, 16, 1024), idesc, (kb | k) != 0);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR) umma_commit_pair(&empty[stage]);
+          else umma_commit(&empty[stage]);
           any = true;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        umma_commit(&acc_full[acc]);
+        if constexpr (PAIR) umma_commit_pair(&acc_full[acc]);
+        else umma_commit(&acc_full[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       if (any) {
-        umma_commit(drain);
+        if constexpr (PAIR) umma_commit_pair(drain);
+        else umma_commit(drain);
         mbar_wait(drain, 0);
       }
     }
@@ -184,11 +217,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool out_bf16 = p.epi == int(Epi::kSiluSplit) || !p.io_fp32;
     const int step = out_bf16 ? 64 : 32;   // columns per 128-byte box row
     uint32_t acc = 0, acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int64_t t = t0; t < total; t += t_step) {
       if (*abort_flag) break;
       const int64_t mt = t / n_tiles;
       const int nt = int(t % n_tiles);
-      const int64_t grow = mt * 128 + row;
+      const int64_t row0 = mt * kTileM + int64_t(rank) * 128;   // this CTA's first row
+      const int64_t grow = row0 + row;
       const bool valid = grow < p.M;   // rows past M are computed on zeros and clipped by the store
       // fp32 residual: the loads of a chunk are issued one chunk ahead (the
       // first chunk's before the wait for the accumulator), so that their
@@ -234,7 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           fence_proxy_async_smem();   // make the stores visible to the TMA unit
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tma_out, box, col0, int32_t(mt * 128 + q * 32));
+            tma_store_2d(tma_out, box, col0, int32_t(row0 + q * 32));
             bulk_commit_group();
             bulk_wait_group_read0();   // the box is refilled by the next step
           }
@@ -253,7 +287,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tma_out2, box, col0, int32_t(mt * 128 + q * 32));
+              tma_store_2d(tma_out2, box, col0, int32_t(row0 + q * 32));
               bulk_commit_group();
               bulk_wait_group_read0();
             }
@@ -305,33 +339,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_proxy_async_smem();   // make the stores visible to the TMA unit
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tma_out, box, col0, int32_t(mt * 128 + q * 32));
+          tma_store_2d(tma_out, box, col0, int32_t(row0 + q * 32));
           bulk_commit_group();
           bulk_wait_group_read0();   // the box is refilled by the next step
         }
         __syncwarp();
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      if constexpr (PAIR) {
+        __syncwarp();
+        if (lane == 0) arrive_leader(leader(&acc_empty[acc]));
+      } else {
+        mbar_arrive(&acc_empty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
   }
 
+  tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the leader's products read the peer's memory until done
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.error, HSTU_DEVERR_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 2 * BN);
+    else tmem_dealloc(tmem_base, 2 * BN);
   }
 }
 
 template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
+                   const __grid_constant__ CUtensorMap tma_b,
+                   const __grid_constant__ CUtensorMap tma_out,
+                   const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
+  gemm_body<BN, false>(&tma_a, &tma_b, &tma_out, &tma_out2, p);
+}
+
+// 256 x 256 output tiles on a cluster of two CTAs (M = 256 cta_group::2
+// products): each SM brings in half of every B tile, so the L2 -> shared
+// memory operand stream per output element is a third smaller than with
+// 128 x 256 tiles.  The loads are plain (no multicast).
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
+                        const __grid_constant__ CUtensorMap tma_b,
+                        const __grid_constant__ CUtensorMap tma_out,
+                        const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
+  gemm_body<256, true>(&tma_a, &tma_b, &tma_out, &tma_out2, p);
+}
+
+template <int BN, bool PAIR>
 cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
-  using L = GemmLayout<BN>;
+  using L = GemmLayout<BN, PAIR>;
   CUtensorMap ta, tb, to, to2;
   if (!make_tmap_2d_bf16(&ta, a.a, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K) * 2, kBK, 128))
     return cudaErrorInvalidValue;
-  if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK, BN))
+  if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK,
+                         PAIR ? BN / 2 : BN))
     return cudaErrorInvalidValue;
   // output boxes: 32 rows x 128 bytes (64 bf16 or 32 fp32 columns)
   const bool out_f32 = a.epi == Epi::kBiasResidual && a.io_fp32;
@@ -346,7 +410,9 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
                                       uint64_t(a.N) * 2, 32, 32))
     return cudaErrorInvalidValue;
   static std::atomic<uint64_t> smem_set{0};
-  const cudaError_t e = smem_opt_in(gemm_tc_kernel<BN>, int(L::kSmemBytes), smem_set);
+  const cudaError_t e =
+      PAIR ? smem_opt_in(gemm_tc_pair_kernel, int(L::kSmemBytes), smem_set)
+           : smem_opt_in(gemm_tc_kernel<BN>, int(L::kSmemBytes), smem_set);
   if (e != cudaSuccess) return e;
   GemmParams p;
   p.M = a.M;
@@ -360,9 +426,16 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   p.out_bf16 = copy ? 1 : 0;
   p.wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimit;
   p.error = error;
-  const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
-  const int grid = int(tiles < num_sms ? tiles : num_sms);
-  gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, to2, p);
+  if constexpr (PAIR) {
+    const int64_t tiles = ((a.M + 255) / 256) * (a.N / BN);
+    const int64_t clusters = tiles < num_sms / 2 ? tiles : int64_t(num_sms / 2);
+    gemm_tc_pair_kernel<<<unsigned(2 * clusters), kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to,
+                                                                                     to2, p);
+  } else {
+    const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
+    const int grid = int(tiles < num_sms ? tiles : num_sms);
+    gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, to2, p);
+  }
   return cudaGetLastError();
 }
 
@@ -371,8 +444,13 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
 cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
   if (a.M <= 0) return cudaSuccess;
   if (a.K % kBK != 0 || a.N % 128 != 0) return cudaErrorInvalidValue;
-  if (a.N % 256 == 0) return launch_bn<256>(a, num_sms, st, error);
-  return launch_bn<128>(a, num_sms, st, error);
+  // f1 (the SiLU-split epilogue, N = 4d) on CTA pairs when there are tiles
+  // for every pair of SMs
+  if (a.N % 256 == 0 && a.epi == Epi::kSiluSplit && num_sms >= 2 &&
+      ((a.M + 255) / 256) * (a.N / 256) >= num_sms / 2)
+    return launch_bn<256, true>(a, num_sms, st, error);
+  if (a.N % 256 == 0) return launch_bn<256, false>(a, num_sms, st, error);
+  return launch_bn<128, false>(a, num_sms, st, error);
 }
 
 }  // namespace hstu
