@@ -48,12 +48,14 @@ struct GemmParams {
 // products (each CTA holds 128 rows of A and BN / 2 rows of the B tile).
 template <int BN, bool PAIR>
 struct GemmLayout {
-  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kStages = PAIR ? 5 : 4;
   static constexpr uint32_t kABytes = 128 * kBK * 2;
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kOutOffset = kStages * kStageBytes;   // 8 boxes of 4 KB
-  static constexpr uint32_t kBarOffset = kOutOffset + 8 * 4096;
+  // PAIR: 8 boxes of 2 KB of their own for the bf16 copy of an fp32 output
+  static constexpr uint32_t kOut2Offset = kOutOffset + 8 * 4096;
+  static constexpr uint32_t kBarOffset = kOut2Offset + (PAIR ? 8 * 2048 : 0);
   static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
   static_assert(kABytes % 1024 == 0 && kStageBytes % 1024 == 0, "TMA destinations 1024-aligned");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -211,6 +213,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
     const int row = q * 32 + lane;
     const int c_begin = ((warp - 2) >> 2) * (BN / 2);
     uint8_t* box = smem + L::kOutOffset + (warp - 2) * 4096;
+    uint8_t* box2 = smem + L::kOut2Offset + (warp - 2) * 2048;   // PAIR only
     const uint32_t row_addr = smem_u32(box + lane * 128);
     // 16-byte chunk e of this thread's 128-byte box row (128-byte swizzle)
     auto chunk = [&](int e) -> uint32_t { return row_addr + ((e ^ (lane & 7)) << 4); };
@@ -263,20 +266,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
             v[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y + x.y;
             v[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z + x.z;
             v[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w + x.w;
+          }
+          // the boxes went to the TMA unit in the previous step: refill them once
+          // it has read them (the wait overlaps this step's loads and arithmetic)
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
             st_shared_v4(chunk(e), v[4 * e + 0], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          }
-          fence_proxy_async_smem();   // make the stores visible to the TMA unit
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(tma_out, box, col0, int32_t(row0 + q * 32));
-            bulk_commit_group();
-            bulk_wait_group_read0();   // the box is refilled by the next step
-          }
-          __syncwarp();
-          if (p.out_bf16) {
-            // bf16 copy of the 32 fp32 columns: 64-byte box rows, 64-byte swizzle
-            // (16-byte chunk e of row r sits at chunk e ^ ((r / 2) mod 4))
-            const uint32_t row64 = smem_u32(box + lane * 64);
+          // bf16 copy of the 32 fp32 columns: 64-byte box rows, 64-byte swizzle
+          // (16-byte chunk e of row r sits at chunk e ^ ((r / 2) mod 4)); PAIR
+          // stages it in a box of its own, else in the fp32 box once that is read
+          auto stage_bf16 = [&](uint8_t* b) {
+            const uint32_t row64 = smem_u32(b + lane * 64);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               st_shared_v4_u32(row64 + ((e ^ ((lane >> 1) & 3)) << 4),
@@ -284,12 +286,25 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
                                pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
                                pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
                                pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+          };
+          if (PAIR && p.out_bf16) stage_bf16(box2);
+          fence_proxy_async_smem();   // make the stores visible to the TMA unit
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(tma_out, box, col0, int32_t(row0 + q * 32));
+            if (PAIR && p.out_bf16) tma_store_2d(tma_out2, box2, col0, int32_t(row0 + q * 32));
+            bulk_commit_group();
+          }
+          __syncwarp();
+          if (!PAIR && p.out_bf16) {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            stage_bf16(box);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
               tma_store_2d(tma_out2, box, col0, int32_t(row0 + q * 32));
               bulk_commit_group();
-              bulk_wait_group_read0();
             }
             __syncwarp();
           }
@@ -312,6 +327,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
             v[32 * h + 4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w;
           }
         }
+        // the box went to the TMA unit in the previous step: refill it once read
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
         if (p.epi == int(Epi::kSiluSplit)) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -341,7 +359,6 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
         if (lane == 0) {
           tma_store_2d(tma_out, box, col0, int32_t(row0 + q * 32));
           bulk_commit_group();
-          bulk_wait_group_read0();   // the box is refilled by the next step
         }
         __syncwarp();
       }
@@ -354,6 +371,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait_group_read0();   // no store still reads shared memory at exit
+    __syncwarp();
   }
 
   tc_fence_before();
