@@ -46,19 +46,30 @@ struct GemmParams {
 
 // PAIR: a cluster of two CTAs computes a 256 x BN tile with cta_group::2
 // products (each CTA holds 128 rows of A and BN / 2 rows of the B tile).
-template <int BN, bool PAIR>
+// RES (with PAIR, fp32 output + fp32 residual): the residual comes in by TMA
+// through a ring of kResSlots boxes per epilogue warp, two 32-column chunks
+// ahead of use; the output is formed in place in the residual's box and
+// stored from there, so the plain output boxes are not needed.  The epilogue
+// is the bound there, so the operand ring is shorter.
+constexpr int kResSlots = 3;
+template <int BN, bool PAIR, bool RES = false>
 struct GemmLayout {
-  static constexpr int kStages = PAIR ? 5 : 4;
+  static_assert(!RES || PAIR, "the residual ring is laid out for CTA pairs");
+  static constexpr int kStages = RES ? 3 : (PAIR ? 5 : 4);
   static constexpr uint32_t kABytes = 128 * kBK * 2;
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kOutOffset = kStages * kStageBytes;   // 8 boxes of 4 KB
+  static constexpr uint32_t kOutOffset = kStages * kStageBytes;   // 8 boxes of 4 KB (not RES)
   // PAIR: 8 boxes of 2 KB of their own for the bf16 copy of an fp32 output
-  static constexpr uint32_t kOut2Offset = kOutOffset + 8 * 4096;
-  static constexpr uint32_t kBarOffset = kOut2Offset + (PAIR ? 8 * 2048 : 0);
-  static constexpr uint32_t kSmemBytes = kBarOffset + 256 + 1024;   // + alignment slack
+  static constexpr uint32_t kOut2Offset = kOutOffset + (RES ? 0 : 8 * 4096);
+  static constexpr uint32_t kResOffset = kOut2Offset + (PAIR ? 8 * 2048 : 0);
+  static constexpr uint32_t kBarOffset = kResOffset + (RES ? 8 * kResSlots * 4096 : 0);
+  static constexpr uint32_t kSmemBytes = kBarOffset + 512 + 1024;   // + alignment slack
   static_assert(kABytes % 1024 == 0 && kStageBytes % 1024 == 0, "TMA destinations 1024-aligned");
+  static_assert(kOut2Offset % 1024 == 0 && kResOffset % 1024 == 0, "box alignment");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  // mbarriers: the ring (2 kStages), 4 accumulator, drain, 8 x kResSlots residual; two words
+  static_assert((2 * kStages + 5 + 8 * kResSlots) * 8 + 8 <= 512, "barrier block");
 };
 
 // SiLU(v) = v / (1 + e^-v) with the hardware exp2 and reciprocal (relative
@@ -68,11 +79,11 @@ __device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + _
 
 constexpr int kGemmThreads = 320;
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool RES>
 __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtensorMap* tma_b,
                                           const CUtensorMap* tma_out, const CUtensorMap* tma_out2,
-                                          const GemmParams& p) {
-  using L = GemmLayout<BN, PAIR>;
+                                          const CUtensorMap* tma_res, const GemmParams& p) {
+  using L = GemmLayout<BN, PAIR, RES>;
   constexpr int kStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -82,7 +93,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
   uint64_t* acc_full = empty + kStages;   // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* res_full = drain + 1;         // [8 warps][kResSlots] (RES)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_full + 8 * kResSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -102,6 +114,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
       mbar_init(&acc_empty[a], PAIR ? 16 : 256);   // PAIR: each epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < 8 * kResSlots; ++r) mbar_init(&res_full[r], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -220,6 +233,107 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
     const bool out_bf16 = p.epi == int(Epi::kSiluSplit) || !p.io_fp32;
     const int step = out_bf16 ? 64 : 32;   // columns per 128-byte box row
     uint32_t acc = 0, acc_phase = 0;
+    if constexpr (RES) {
+      // fp32 output = acc + bias + the fp32 residual, 32 columns per chunk; the
+      // warp's chunk k is tile t0 + (k / kChunks) t_step, columns c_begin + 32 (k % kChunks)
+      constexpr int kChunks = (BN / 2) / 32;
+      const int wi = warp - 2;
+      uint8_t* rbox = smem + L::kResOffset + wi * kResSlots * 4096;
+      uint64_t* rbar = res_full + wi * kResSlots;
+      int64_t issued = -1;   // the last chunk whose residual load was issued (lane 0)
+      auto issue_res = [&](int64_t k) {
+        const int64_t tt = t0 + (k / kChunks) * t_step;
+        if (tt >= total) return;
+        const int cc = c_begin + 32 * int(k % kChunks);
+        const int slot = int(k % kResSlots);
+        mbar_arrive_expect_tx(&rbar[slot], 4096);
+        tma_load_2d(rbox + slot * 4096, tma_res, &rbar[slot], int(tt % n_tiles) * BN + cc,
+                    int32_t((tt / n_tiles) * kTileM + int64_t(rank) * 128 + q * 32));
+        issued = k;
+      };
+      if (lane == 0) {
+        issue_res(0);
+        issue_res(1);
+      }
+      int64_t k = 0;
+      bool ok = true;
+      for (int64_t t = t0; ok && t < total; t += t_step) {
+        if (*abort_flag) break;
+        const int64_t mt = t / n_tiles;
+        const int nt = int(t % n_tiles);
+        const int64_t row0 = mt * kTileM + int64_t(rank) * 128;   // this CTA's first row
+        if (!mbar_wait(&acc_full[acc], acc_phase, p.wait_limit)) { *abort_flag = 1; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + BN / 2; c += 32, ++k) {
+          const int col0 = nt * BN + c;
+          const int slot = int(k % kResSlots);
+          uint32_t r[32];
+          tmem_ld32(tmem_base + acc * BN + c + (uint32_t(q * 32) << 16), r);
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(&rbar[slot], uint32_t(k / kResSlots) & 1, p.wait_limit));
+          tmem_ld_wait();
+          if (!ok) {
+            *abort_flag = 1;
+            break;
+          }
+          // the residual's box row of this thread (128-byte swizzle), overwritten by the output
+          const uint32_t xrow = smem_u32(rbox + slot * 4096 + lane * 128);
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t at = xrow + ((e ^ (lane & 7)) << 4);
+            const float4 x = ld_shared_v4(at);
+            const float4 bb = __ldg(b4 + e);
+            v[4 * e + 0] = __uint_as_float(r[4 * e + 0]) + bb.x + x.x;
+            v[4 * e + 1] = __uint_as_float(r[4 * e + 1]) + bb.y + x.y;
+            v[4 * e + 2] = __uint_as_float(r[4 * e + 2]) + bb.z + x.z;
+            v[4 * e + 3] = __uint_as_float(r[4 * e + 3]) + bb.w + x.w;
+            st_shared_v4(at, v[4 * e + 0], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+          // the previous chunk's stores have read their boxes: its residual slot
+          // takes chunk k + 2, and the bf16 box is refilled
+          if (lane == 0) {
+            bulk_wait_group_read0();
+            issue_res(k + 2);
+          }
+          __syncwarp();
+          if (p.out_bf16) {
+            // 64-byte box rows, 64-byte swizzle (16-byte chunk e of row r sits at
+            // chunk e ^ ((r / 2) mod 4))
+            const uint32_t row64 = smem_u32(box2 + lane * 64);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              st_shared_v4_u32(row64 + ((e ^ ((lane >> 1) & 3)) << 4),
+                               pack_bf16x2(v[8 * e + 0], v[8 * e + 1]),
+                               pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                               pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                               pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+          }
+          fence_proxy_async_smem();   // make the stores visible to the TMA unit
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(tma_out, rbox + slot * 4096, col0, int32_t(row0 + q * 32));
+            if (p.out_bf16) tma_store_2d(tma_out2, box2, col0, int32_t(row0 + q * 32));
+            bulk_commit_group();
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_leader(leader(&acc_empty[acc]));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      // no residual load lands and no store reads shared memory after the exit
+      if (lane == 0) {
+        for (int64_t kk = k; kk <= issued; ++kk)
+          mbar_wait(&rbar[kk % kResSlots], uint32_t(kk / kResSlots) & 1, p.wait_limit);
+        bulk_wait_group_read0();
+      }
+      __syncwarp();
+    } else {
     for (int64_t t = t0; t < total; t += t_step) {
       if (*abort_flag) break;
       const int64_t mt = t / n_tiles;
@@ -373,6 +487,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap* tma_a, const CUtens
     }
     if (lane == 0) bulk_wait_group_read0();   // no store still reads shared memory at exit
     __syncwarp();
+    }
   }
 
   tc_fence_before();
@@ -391,26 +506,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
                    const __grid_constant__ CUtensorMap tma_b,
                    const __grid_constant__ CUtensorMap tma_out,
-                   const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
-  gemm_body<BN, false>(&tma_a, &tma_b, &tma_out, &tma_out2, p);
+                   const __grid_constant__ CUtensorMap tma_out2,
+                   const __grid_constant__ CUtensorMap tma_res, const GemmParams p) {
+  gemm_body<BN, false, false>(&tma_a, &tma_b, &tma_out, &tma_out2, &tma_res, p);
 }
 
 // 256 x 256 output tiles on a cluster of two CTAs (M = 256 cta_group::2
 // products): each SM brings in half of every B tile, so the L2 -> shared
 // memory operand stream per output element is a third smaller than with
 // 128 x 256 tiles.  The loads are plain (no multicast).
+// RES: the fp32-residual epilogue with the residual brought in by TMA.
+template <bool RES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                         const __grid_constant__ CUtensorMap tma_b,
                         const __grid_constant__ CUtensorMap tma_out,
-                        const __grid_constant__ CUtensorMap tma_out2, const GemmParams p) {
-  gemm_body<256, true>(&tma_a, &tma_b, &tma_out, &tma_out2, p);
+                        const __grid_constant__ CUtensorMap tma_out2,
+                        const __grid_constant__ CUtensorMap tma_res, const GemmParams p) {
+  gemm_body<256, true, RES>(&tma_a, &tma_b, &tma_out, &tma_out2, &tma_res, p);
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool RES = false>
 cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* error) {
-  using L = GemmLayout<BN, PAIR>;
-  CUtensorMap ta, tb, to, to2;
+  using L = GemmLayout<BN, PAIR, RES>;
+  CUtensorMap ta, tb, to, to2, tr;
   if (!make_tmap_2d_bf16(&ta, a.a, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K) * 2, kBK, 128))
     return cudaErrorInvalidValue;
   if (!make_tmap_2d_bf16(&tb, a.b, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, kBK,
@@ -428,9 +547,13 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   if (copy && !make_tmap_2d_bf16_sw64(&to2, a.out_bf16, uint64_t(a.N), uint64_t(a.M),
                                       uint64_t(a.N) * 2, 32, 32))
     return cudaErrorInvalidValue;
+  tr = to;   // unused unless RES: the fp32 residual in the output's box format
+  if (RES && !make_tmap_2d_f32_sw128(&tr, a.residual, uint64_t(a.N),
+                                     uint64_t(a.M), uint64_t(a.N) * 4, 32, 32))
+    return cudaErrorInvalidValue;
   static std::atomic<uint64_t> smem_set{0};
   const cudaError_t e =
-      PAIR ? smem_opt_in(gemm_tc_pair_kernel, int(L::kSmemBytes), smem_set)
+      PAIR ? smem_opt_in(gemm_tc_pair_kernel<RES>, int(L::kSmemBytes), smem_set)
            : smem_opt_in(gemm_tc_kernel<BN>, int(L::kSmemBytes), smem_set);
   if (e != cudaSuccess) return e;
   GemmParams p;
@@ -448,12 +571,12 @@ cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t st, int32_t* 
   if constexpr (PAIR) {
     const int64_t tiles = ((a.M + 255) / 256) * (a.N / BN);
     const int64_t clusters = tiles < num_sms / 2 ? tiles : int64_t(num_sms / 2);
-    gemm_tc_pair_kernel<<<unsigned(2 * clusters), kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to,
-                                                                                     to2, p);
+    gemm_tc_pair_kernel<RES><<<unsigned(2 * clusters), kGemmThreads, L::kSmemBytes, st>>>(
+        ta, tb, to, to2, tr, p);
   } else {
     const int64_t tiles = ((a.M + 127) / 128) * (a.N / BN);
     const int grid = int(tiles < num_sms ? tiles : num_sms);
-    gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, to2, p);
+    gemm_tc_kernel<BN><<<grid, kGemmThreads, L::kSmemBytes, st>>>(ta, tb, to, to2, tr, p);
   }
   return cudaGetLastError();
 }
@@ -466,8 +589,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int3
   // CTA pairs when there are 256 x 256 tiles for every pair of SMs (measured
   // on one c3 layer: f1 7.5% and f2 4% faster than 128 x 256 tiles)
   if (a.N % 256 == 0 && num_sms >= 2 &&
-      ((a.M + 255) / 256) * (a.N / 256) >= num_sms / 2)
+      ((a.M + 255) / 256) * (a.N / 256) >= num_sms / 2) {
+    if (a.epi == Epi::kBiasResidual && a.io_fp32) return launch_bn<256, true, true>(a, num_sms, st, error);
     return launch_bn<256, true>(a, num_sms, st, error);
+  }
   if (a.N % 256 == 0) return launch_bn<256, false>(a, num_sms, st, error);
   return launch_bn<128, false>(a, num_sms, st, error);
 }
