@@ -76,6 +76,12 @@ def _check_layer(w, batch, res):
     # bf16 tensor-core path
     assert rel_err(res["Y"], ref["Y"]) <= 2e-2
     uvqk = np.concatenate([ref["U"], ref["V"], ref["Q"], ref["K"]], axis=1)
+    if w.storage == "fp32":
+        # an fp32 residual stream with bf16 operands: f1's GEMM reads bf16(X), so
+        # its outputs are compared with f1 evaluated on that input (the residual
+        # and everything checked above keep the exact fp32 X)
+        Xb = oracle_inputs(batch, "bf16")
+        uvqk = np.concatenate(oracle.f1_split(Xb, p["w1"], p["b1"], d), axis=1)
     r = np.sqrt(np.mean(uvqk ** 2))
     assert np.all(np.abs(res["UVQK"] - uvqk) <= 2.0 ** -8 * np.abs(uvqk) + 1e-3 * r)
     O_tf, O_abs = teacher_forced_attention(res["UVQK"], batch, cfg, p, with_abs=True)
@@ -105,6 +111,23 @@ def test_fp32_path_with_strong_attention():
                                  rab_scale=1.0, random_affine=True, feature_scale=1.0,
                                  timestamp_gap=600.0)
     res = gpu_run(batch, "fp32", "fp32", d=64, H=2, n_norm=0, mask="causal")
+    _check_layer(w, batch, res)
+
+
+@pytest.mark.parametrize("lengths", [[1800, 1700, 1220], [1800, 1700, 1333]])
+def test_fp32_residual_stream_ragged_pair_tiles(lengths):
+    """fp32 residual stream, bf16 compute, d 1024 (c3's precision and width) at
+    ragged token counts large enough for the CTA-pair GEMMs (f2 takes its
+    residual by TMA): 4720 tokens leave the second CTA of the last 256-row tile
+    wholly past T, 4833 partly."""
+    d, H = 1024, 8
+    batch = wl.make_custom_batch(lengths, d, H, seed=sum(lengths), weight_scale=0.03,
+                                 rab_scale=1.0, random_affine=True, timestamp_gap=900.0)
+    w = wl.Workload("fp32 residual, ragged", 98, num_users=len(lengths), d_model=d, num_heads=H,
+                    head_dim=128, num_layers=1, storage="fp32", compute="bf16", pos_buckets=129,
+                    pos_clamp=128, time_buckets=128, time_log_div=0.301, n_norm=2048,
+                    mask="causal", lengths="custom", features="normal_1")
+    res = gpu_run(batch, "fp32", "bf16", d=d, H=H, n_norm=2048, mask="causal")
     _check_layer(w, batch, res)
 
 
