@@ -593,7 +593,9 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, int num_sms, cudaStream_t st, int3
     if (a.epi == Epi::kBiasResidual && a.io_fp32) return launch_bn<256, true, true>(a, num_sms, st, error);
     return launch_bn<256, true>(a, num_sms, st, error);
   }
-  if (a.N % 256 == 0) return launch_bn<256, false>(a, num_sms, st, error);
+  // 128 x 256 tiles when they fill a wave, else 128 x 128 (twice the tiles)
+  if (a.N % 256 == 0 && ((a.M + 127) / 128) * (a.N / 256) >= num_sms)
+    return launch_bn<256, false>(a, num_sms, st, error);
   return launch_bn<128, false>(a, num_sms, st, error);
 }
 
