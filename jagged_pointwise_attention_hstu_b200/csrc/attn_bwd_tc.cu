@@ -40,7 +40,10 @@
 // every position bucket is the clamped one and each row meets one time bucket
 // (the common case far from the diagonal), the bias is a per-row constant and
 // the bias gradients are per-row sums; otherwise every pair takes the mask,
-// the position bucket and the exact time bucket.
+// the position bucket and the exact time bucket.  Position-bucket gradients of
+// rows at their own positions are summed along the tile diagonals in three
+// register slots per lane over a half tile; rows at one position (M-FALCON
+// candidates) sum the columns with a 16-shuffle butterfly.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -183,6 +186,40 @@ __device__ __forceinline__ void store_box(uint32_t taddr, uint8_t* box, const CU
     bulk_wait_group_read0();
   }
   __syncwarp();
+}
+
+// Adds v to the position-bucket gradient of relative position p (clamped); the
+// clamped bucket's share goes to the row's register sum instead.
+__device__ __forceinline__ void add_pos_grad(float* s_gpos, int p, int clamp, float v, float& acc_c) {
+  const int b = p < 0 ? 0 : (p > clamp ? clamp : p);
+  if (b == clamp) acc_c += v;
+  else if (v != 0.0f) red_add_shared(s_gpos + b, v);
+}
+
+// Column sums of a warp's 32 x 16 chunk: after the butterfly, lane l (l even)
+// holds the sum over all 32 lanes of column (l >> 1) & 15 (16 shuffles
+// instead of one 5-step reduction per column).
+__device__ __forceinline__ float column_sums16(const float (&v)[16], int lane) {
+  float a[8], b[4], c[2];
+  const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4, h1 = lane & 2;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float send = h4 ? v[k] : v[k + 8];
+    a[k] = (h4 ? v[k + 8] : v[k]) + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float send = h3 ? a[k] : a[k + 4];
+    b[k] = (h3 ? a[k + 4] : a[k]) + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float send = h2 ? b[k] : b[k + 2];
+    c[k] = (h2 ? b[k + 2] : b[k]) + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  const float send = h1 ? c[0] : c[1];
+  float s = (h1 ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, send, 2);
+  return s + __shfl_xor_sync(0xffffffffu, s, 1);
 }
 
 // ================================================================ dq kernel
@@ -462,6 +499,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         jm += 64 * g;
         const float ht0 = s_rt[tb0], ht1 = s_rt[tb1];
         float acc_t = 0.0f, acc_t1 = 0.0f;
+        // diagonal sums over the half tile: slot w holds relative position
+        // pos0 - (kb + 64 g) + lane - 32 w
+        float dg0 = 0.0f, dg1 = 0.0f, dg2 = 0.0f;
         // the next chunk's tensor-memory loads run under this chunk's reductions
         uint32_t rs[16], ra[16];
         tmem_ld16(tS + tcol, rs);
@@ -489,32 +529,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_ld16(tdA + tcol + 16 * (c + 1), ra);
           }
           if (diag) {
+            // lane l takes pair (row (l + 16 c + e) mod 32, column e) of the chunk:
+            // its relative position is pos0 - (kb + 64 g) + l - 32 w, w the wrap count
+            // (chunks 0 and 1 wrap from slot 0 into slot 1, chunks 2 and 3 from 1 into 2)
+            const int sh = lane + 16 * (c & 1);
             float acc_a = 0.0f, acc_b = 0.0f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float v = __shfl_sync(0xffffffffu, dsv[e], (lane + e) & 31);
-              if (lane + e < 32) acc_a += v; else acc_b += v;
+              const float v = __shfl_sync(0xffffffffu, dsv[e], (sh + e) & 31);
+              if (sh + e < 32) acc_a += v; else acc_b += v;
             }
-            const int da = pos0 + lane - (kb + jr0);
-            const int db = da - 32;
-            const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
-            const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
-            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) red_add_shared(s_gpos + ba, acc_a);
-            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) red_add_shared(s_gpos + bb, acc_b);
+            if (c < 2) {
+              dg0 += acc_a;
+              dg1 += acc_b;
+            } else {
+              dg1 += acc_a;
+              dg2 += acc_b;
+            }
           } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float v = dsv[e];
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-              if (lane == e && v != 0.0f) {
-                const int dp = pos0 - (kb + jr0 + e);
-                const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-                if (b == clamp) acc_c += v; else red_add_shared(s_gpos + b, v);
-              }
-            }
+            const float v = column_sums16(dsv, lane);
+            if ((lane & 1) == 0)
+              add_pos_grad(s_gpos, pos0 - (kb + jr0 + ((lane >> 1) & 15)), clamp, v, acc_c);
           }
           tmem_ld_wait();
+        }
+        if (diag) {
+          const int p0 = pos0 - (kb + 64 * g) + lane;
+          add_pos_grad(s_gpos, p0, clamp, dg0, acc_c);
+          add_pos_grad(s_gpos, p0 - 32, clamp, dg1, acc_c);
+          add_pos_grad(s_gpos, p0 - 64, clamp, dg2, acc_c);
         }
         const float wsum = warp_sum(acc_t);
         if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
@@ -582,6 +625,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int pos_rel = min(max(pos - kb, -1), clamp + 129);
         int run_b = -1;
         float run_acc = 0.0f;
+        float dg0 = 0.0f, dg1 = 0.0f, dg2 = 0.0f;   // diagonal sums, as on the two-bucket path
         uint32_t rs[16], ra[16];
         tmem_ld16(tS + tcol, rs);
         tmem_ld16(tdA + tcol, ra);
@@ -635,33 +679,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           // position buckets
           if (diag) {
-            // pair (lane l + e, column e) has position pos0 + l - (kb + jr0): lane l
-            // gathers them (and the wrapped ones, 32 positions lower)
+            // as on the two-bucket path: lane l takes pair (row (l + 16 c + e) mod 32,
+            // column e) of the chunk, summed into slot w of its relative position
+            // (chunks 0 and 1 wrap from slot 0 into slot 1, chunks 2 and 3 from 1 into 2)
+            const int sh = lane + 16 * (c & 1);
             float acc_a = 0.0f, acc_b = 0.0f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float v = __shfl_sync(0xffffffffu, dsv[e], (lane + e) & 31);
-              if (lane + e < 32) acc_a += v; else acc_b += v;
+              const float v = __shfl_sync(0xffffffffu, dsv[e], (sh + e) & 31);
+              if (sh + e < 32) acc_a += v; else acc_b += v;
             }
-            const int da = pos0 + lane - (kb + jr0);
-            const int db = da - 32;
-            const int ba = da < 0 ? 0 : (da > clamp ? clamp : da);
-            const int bb = db < 0 ? 0 : (db > clamp ? clamp : db);
-            if (ba == clamp) acc_c += acc_a; else if (acc_a != 0.0f) red_add_shared(s_gpos + ba, acc_a);
-            if (bb == clamp) acc_c += acc_b; else if (acc_b != 0.0f) red_add_shared(s_gpos + bb, acc_b);
+            if (c < 2) {
+              dg0 += acc_a;
+              dg1 += acc_b;
+            } else {
+              dg1 += acc_a;
+              dg2 += acc_b;
+            }
           } else if (col) {
-            // one position per column: the column sums, lane e adds column e
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float v = dsv[e];
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-              if (lane == e && v != 0.0f) {
-                const int dp = pos0 - (kb + jr0 + e);
-                const int b = dp < 0 ? 0 : (dp > clamp ? clamp : dp);
-                if (b == clamp) acc_c += v; else red_add_shared(s_gpos + b, v);
-              }
-            }
+            // one position per column (M-FALCON candidates): the column sums
+            const float v = column_sums16(dsv, lane);
+            if ((lane & 1) == 0)
+              add_pos_grad(s_gpos, pos0 - (kb + jr0 + ((lane >> 1) & 15)), clamp, v, acc_c);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -674,6 +713,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_wait();
         }
         if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
+        if (diag) {
+          const int p0 = pos0 - (kb + 64 * g) + lane;
+          add_pos_grad(s_gpos, p0, clamp, dg0, acc_c);
+          add_pos_grad(s_gpos, p0 - 32, clamp, dg1, acc_c);
+          add_pos_grad(s_gpos, p0 - 64, clamp, dg2, acc_c);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
