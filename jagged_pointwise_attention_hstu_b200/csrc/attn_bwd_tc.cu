@@ -165,6 +165,23 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Adds each lane's v (where pred holds and v != 0) to table[b], b per lane,
+// with one shared add per distinct bucket: the lanes of a bucket are summed
+// with shuffles first.  Shared-memory float adds from many lanes to one word
+// are serialised by the hardware, and neighbouring rows mostly share a time
+// bucket.  Every lane of the warp must call it.
+__device__ __forceinline__ void warp_bucket_add(float* table, int b, float v, bool pred, int lane) {
+  unsigned todo = __ballot_sync(0xffffffffu, pred && v != 0.0f);
+  while (todo != 0u) {
+    const int leader = __ffs(todo) - 1;
+    const int bl = __shfl_sync(0xffffffffu, b, leader);
+    const bool mine = ((todo >> lane) & 1u) != 0u && b == bl;
+    const float s = warp_sum(mine ? v : 0.0f);
+    if (lane == leader) red_add_shared(table + bl, s);
+    todo &= ~__ballot_sync(0xffffffffu, mine);
+  }
+}
+
 // Stages 32 rows x 32 fp32 columns of tensor memory (this warp's lanes) into a
 // 128-byte-swizzled 4 KB box and writes it with a TMA store at (x, y).
 __device__ __forceinline__ void store_box(uint32_t taddr, uint8_t* box, const CUtensorMap* m,
@@ -559,13 +576,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           add_pos_grad(s_gpos, p0 - 32, clamp, dg1, acc_c);
           add_pos_grad(s_gpos, p0 - 64, clamp, dg2, acc_c);
         }
-        const float wsum = warp_sum(acc_t);
-        if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
-          if (lane == 0 && wsum != 0.0f) red_add_shared(s_gtime + tb0, wsum);
-        } else if (acc_t != 0.0f) {
-          red_add_shared(s_gtime + tb0, acc_t);
-        }
-        if (acc_t1 != 0.0f) red_add_shared(s_gtime + tb1, acc_t1);
+        warp_bucket_add(s_gtime, tb0, acc_t, true, lane);
+        warp_bucket_add(s_gtime, tb1, acc_t1, true, lane);
       } else if (fast) {
         // every pair visible, clamped position, one time bucket per row; the
         // tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
@@ -609,12 +621,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_wait();
         }
         acc_c += acc;   // the position bucket is the clamped one for every pair here
-        const float wsum = warp_sum(acc);
-        if (__all_sync(0xffffffffu, tb0 == __shfl_sync(0xffffffffu, tb0, 0))) {
-          if (lane == 0 && wsum != 0.0f) red_add_shared(s_gtime + tb0, wsum);
-        } else if (acc != 0.0f) {
-          red_add_shared(s_gtime + tb0, acc);
-        }
+        warp_bucket_add(s_gtime, tb0, acc, true, lane);
       } else {
         // any visibility: the mask, the position bucket and the exact time bucket
         // of every pair.  The time-bucket gradient is summed along runs of one
@@ -712,7 +719,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tmem_ld_wait();
         }
-        if (run_b >= 0 && run_acc != 0.0f) red_add_shared(s_gtime + run_b, run_acc);
+        warp_bucket_add(s_gtime, run_b, run_acc, run_b >= 0, lane);
         if (diag) {
           const int p0 = pos0 - (kb + 64 * g) + lane;
           add_pos_grad(s_gpos, p0, clamp, dg0, acc_c);
