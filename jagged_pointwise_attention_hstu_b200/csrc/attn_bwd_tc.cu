@@ -241,6 +241,13 @@ __device__ __forceinline__ float column_sums16(const float (&v)[16], int lane) {
 
 // ================================================================ dq kernel
 
+// The time-bucket gradient is kept in kGCopies interleaved copies per CTA
+// (entry b, copy c at b * kGCopies + c): the generic path's per-key flushes of
+// lane l go to copy l mod kGCopies, so neighbouring rows that flush the same
+// bucket at the same key add to different words (shared float adds to one
+// word serialise); the copies are summed once at the end.
+constexpr int kGCopies = 8;
+
 template <int HD>
 struct DqLayout {
   static constexpr int NS = HD == 128 ? 2 : 3;    // K / V ring stages
@@ -252,8 +259,8 @@ struct DqLayout {
   static constexpr uint32_t kKts = kV + NS * kTile;         // int64 [NS][128]
   static constexpr uint32_t kThr = kKts + NS * 1024;        // int64 [256]
   static constexpr uint32_t kRt = kThr + 2048;              // float [256]
-  static constexpr uint32_t kGtime = kRt + 1024;            // float [256]
-  static constexpr uint32_t kAny = kGtime + 1024;           // int4 [128]
+  static constexpr uint32_t kGtime = kRt + 1024;            // float [256][kGCopies]
+  static constexpr uint32_t kAny = kGtime + 1024 * kGCopies;   // int4 [128]
   static constexpr uint32_t kBars = kAny + 2048;
   static constexpr uint32_t kGpos = kBars + 256;            // float [clamp + 1], then the rab_pos copy
   static __host__ __device__ constexpr uint32_t rp_offset(int clamp) {
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int t = threadIdx.x - 128;
     load_tables(p, t, s_thr, s_rt, s_any);
     if (p.rp_smem) load_rp(p, t, s_rp);
-    s_gtime[t] = 0.0f;
+    for (int k = t; k < 256 * kGCopies; k += 256) s_gtime[k] = 0.0f;
     for (int k = t; k <= clamp; k += 256) s_gpos[k] = 0.0f;
   }
   tc_fence_before();
@@ -576,8 +583,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           add_pos_grad(s_gpos, p0 - 32, clamp, dg1, acc_c);
           add_pos_grad(s_gpos, p0 - 64, clamp, dg2, acc_c);
         }
-        warp_bucket_add(s_gtime, tb0, acc_t, true, lane);
-        warp_bucket_add(s_gtime, tb1, acc_t1, true, lane);
+        warp_bucket_add(s_gtime, tb0 * kGCopies, acc_t, true, lane);
+        warp_bucket_add(s_gtime, tb1 * kGCopies, acc_t1, true, lane);
       } else if (fast) {
         // every pair visible, clamped position, one time bucket per row; the
         // tensor-memory loads of chunk c + 1 overlap the arithmetic of chunk c
@@ -621,7 +628,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld_wait();
         }
         acc_c += acc;   // the position bucket is the clamped one for every pair here
-        warp_bucket_add(s_gtime, tb0, acc, true, lane);
+        warp_bucket_add(s_gtime, tb0 * kGCopies, acc, true, lane);
       } else {
         // any visibility: the mask, the position bucket and the exact time bucket
         // of every pair.  The time-bucket gradient is summed along runs of one
@@ -680,7 +687,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const bool next = tbv[e] >= 0 && tbv[e] != run_b;
-            red_add_shared_if(next && run_b >= 0, s_gtime + (run_b < 0 ? 0 : run_b), run_acc);
+            red_add_shared_if(next && run_b >= 0,
+                              s_gtime + (run_b < 0 ? 0 : run_b) * kGCopies + (lane & (kGCopies - 1)),
+                              run_acc);
             run_acc = next ? dsv[e] : run_acc + dsv[e];
             run_b = next ? tbv[e] : run_b;
           }
@@ -719,7 +728,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tmem_ld_wait();
         }
-        warp_bucket_add(s_gtime, run_b, run_acc, run_b >= 0, lane);
+        warp_bucket_add(s_gtime, run_b * kGCopies, run_acc, run_b >= 0, lane);
         if (diag) {
           const int p0 = pos0 - (kb + 64 * g) + lane;
           add_pos_grad(s_gpos, p0, clamp, dg0, acc_c);
@@ -759,7 +768,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (gv != 0.0f) atomicAdd(p.d_rab_pos + k, gv);
     }
     if (t < nb) {
-      const float gv = s_gtime[t];
+      float gv = 0.0f;
+#pragma unroll
+      for (int c = 0; c < kGCopies; ++c) gv += s_gtime[t * kGCopies + c];
       if (gv != 0.0f) atomicAdd(p.d_rab_time + t, gv);
     }
   }
